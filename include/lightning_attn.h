@@ -1,0 +1,113 @@
+/*
+ * lightning_attn.h -- C ABI of the B200 (sm_100a) Lightning Attention library.
+ *
+ * The operation (one independent problem per batch row b and head h):
+ *
+ *     o_t = sum_{s <= t} exp(-lambda_h * (t - s)) * (q_t . k_s) * v_s
+ *
+ * i.e. causal linear attention with a fixed per-head exponential decay and no
+ * normaliser, no softmax and no in-kernel scale.  Sources for the operation:
+ *   - "MiniMax-M1" model entry (archdb), field "Configuration of the linear / SSM
+ *     layers": Lightning attention with a per-head exponential decay
+ *     (ALiBi-style slopes) and a 128x128 state per head.
+ *   - same entry, positional-scheme field: Lightning layers use a fixed per-head
+ *     decay and no RoPE, so position enters only through the decay.
+ *   - "MiniMax-01" (redeep.blog), section "What Makes 1M Context Hard": a
+ *     linear-complexity variant that replaces softmax attention.
+ *   - Lightning Attention news article (cocoloop), section "El enfoque de
+ *     Lightning Attention": complexity reduced from O(n^2) to about O(n).
+ * lambda_h is the decay RATE (slope); the per-token factor is gamma_h =
+ * exp(-lambda_h), so lambda_h = 0 is plain causal linear attention.  The
+ * diagonal s = t is included.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     never frees them and keeps no reference after the call returns.
+ *   - Layout is head-major and contiguous: q, k are [B][H][N][D], v is
+ *     [B][H][N][E], out is [B][H][N][E] (decode: N is absent).  slopes is a
+ *     float32 device array [H].
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = legacy default stream).  They return a status code and never
+ *     throw, exit or abort.  Argument errors are detected on the host before any
+ *     launch.  A launch failure is reported as LA_ERR_CUDA.
+ *   - Preconditions that are NOT checked (checking them would need a device
+ *     synchronisation): slopes must be finite and >= 0; out must not alias any
+ *     input; decode out must not alias state.
+ *   - Device-side waits are bounded in time.  A wait that runs out sets a
+ *     sticky per-device status word (read it with lightning_attn_device_status)
+ *     and the kernel returns without finishing its outputs.
+ */
+#ifndef LIGHTNING_ATTN_H_
+#define LIGHTNING_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LA_OK = 0,
+  LA_ERR_NULL = 1,        /* a required pointer is NULL                         */
+  LA_ERR_SHAPE = 2,       /* B, H, N < 1, or sizes overflow 64-bit indexing      */
+  LA_ERR_ALIGN = 3,       /* a tensor pointer is not 16-byte aligned            */
+  LA_ERR_UNSUPPORTED = 4, /* D or E outside {64, 128} for this entry point      */
+  LA_ERR_CUDA = 5,        /* a CUDA runtime/driver call or the launch failed    */
+  LA_ERR_TIMEOUT = 6,     /* a bounded device-side wait ran out (see above)     */
+  LA_ERR_WORKSPACE = 7    /* caller workspace missing or too small              */
+} la_status;
+
+/*
+ * Prefill, bf16 inputs, fp32 output.
+ *   q, k : bf16 [B][H][N][D]      v : bf16 [B][H][N][E]
+ *   slopes: fp32 [H], lambda_h    out: fp32 [B][H][N][E] (fully overwritten)
+ * Zero initial state.  D = E = 128 is the supported head geometry (the
+ * "128x128 state per head" of the MiniMax-M1 entry, linear-layer field);
+ * other D, E return LA_ERR_UNSUPPORTED.  Any N >= 1.
+ * Runs on tcgen05 tensor cores (bf16 operands, fp32 accumulation, fp32 state
+ * carried on chip).  Long sequences are split into chunks processed in parallel
+ * with a chained state scan; the scan scratch (about 128 KiB per (b, h)) is
+ * taken with cudaMallocAsync / cudaFreeAsync on `stream`.
+ */
+int lightning_attn_fwd(const void* q, const void* k, const void* v,
+                       const float* slopes, float* out,
+                       int B, int H, int N, int D, int E, void* stream);
+
+/*
+ * Prefill with fp32 inputs and output (same operation and layout as
+ * lightning_attn_fwd, all tensors fp32).  D, E in {64, 128}.  CUDA-core fp32
+ * arithmetic, for callers that need fp32-class accuracy.
+ */
+int lightning_attn_fwd_f32(const float* q, const float* k, const float* v,
+                           const float* slopes, float* out,
+                           int B, int H, int N, int D, int E, void* stream);
+
+/*
+ * One recurrent decode step for B*H independent (b, h) states.
+ *   q, k : bf16 [B][H][D]     v : bf16 [B][H][E]
+ *   state: fp32 [B][H][D][E] (row d, column e), read and written IN PLACE
+ *   out  : fp32 [B][H][E]
+ * Order within the step: state <- exp(-lambda_h) * state + k^T v, then
+ * out = q . state (the updated state; consistent with the inclusive diagonal
+ * of the prefill).  D, E in {64, 128}.
+ */
+int lightning_attn_decode(const void* q, const void* k, const void* v,
+                          float* state, const float* slopes, float* out,
+                          int B, int H, int D, int E, void* stream);
+
+/* Human-readable name of a la_status value (static string, never NULL). */
+const char* lightning_attn_status_string(int status);
+
+/*
+ * Reads the calling thread's current device's sticky device-side status word
+ * (LA_OK or LA_ERR_TIMEOUT) into *status; if reset != 0 clears it.  This call
+ * synchronises with the device.  Returns LA_OK or LA_ERR_NULL / LA_ERR_CUDA.
+ */
+int lightning_attn_device_status(int* status, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIGHTNING_ATTN_H_ */

@@ -1,0 +1,303 @@
+/*
+ * lightning_oracle.c -- plain float64 CPU oracle for Lightning Attention.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke entry point and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or helper with the CUDA library, and the CUDA library never
+ * calls it.  Inputs are the exact values the GPU sees (bf16 bit patterns or
+ * fp32 values, upcast losslessly to double); all arithmetic is double.
+ *
+ * What it computes, for each (b, h) independently (layout [B][H][N][*]):
+ *
+ *     o_t = sum_{s <= t} exp(-lambda_h * (t - s)) * (q_t . k_s) * v_s
+ *
+ * Sources: "MiniMax-M1" model entry (archdb), linear/SSM layer configuration
+ * field (per-head exponential decay, ALiBi-style slopes, 128x128 state per
+ * head) and positional-scheme field (fixed per-head decay, no RoPE);
+ * "MiniMax-01" (redeep.blog), "What Makes 1M Context Hard" (linear-complexity
+ * variant of attention).  lambda_h is read as a decay rate, gamma = exp(-lambda)
+ * as the per-step factor; the sum includes s = t; there is no normaliser.
+ *
+ * Forms (each a plain restatement, no blocking or reordering beyond the form):
+ *   la_oracle_masked     O(N^2 (D+E)) masked sum, the definition itself.
+ *   la_oracle_recurrent  O(N D E) recurrence  S_t = gamma S_{t-1} + k_t^T v_t,
+ *                        o_t = q_t S_t, optionally from an initial state and
+ *                        returning the final state.
+ *   la_oracle_blocked    the same sum split into blocks of `blk` tokens: an
+ *                        intra-block masked term, an inter-block term through
+ *                        the state, and the state carry between blocks.
+ *   la_oracle_recurrent_sampled  the recurrence, emitting o_t only at the
+ *                        given positions (for sequences too long to store).
+ *   la_oracle_decode_step one recurrent step on a given state, in place.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define LA_ORACLE_F32 0
+#define LA_ORACLE_BF16 1
+
+/* One input element as double.  bf16 is the top half of an IEEE binary32. */
+static inline double in_at(const void* p, int64_t i, int dtype) {
+  if (dtype == LA_ORACLE_BF16) {
+    uint32_t bits = ((uint32_t)((const uint16_t*)p)[i]) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+  }
+  return (double)((const float*)p)[i];
+}
+
+/* Copies n consecutive input elements starting at index i0 into dst. */
+static void in_row(double* dst, const void* p, int64_t i0, int64_t n, int dtype) {
+  for (int64_t x = 0; x < n; ++x) dst[x] = in_at(p, i0 + x, dtype);
+}
+
+static int bad_args(const void* q, const void* k, const void* v, const float* slopes,
+                    const void* out, int64_t B, int64_t H, int64_t N, int64_t D, int64_t E) {
+  if (!q || !k || !v || !slopes || !out) return 1;
+  if (B < 1 || H < 1 || N < 0 || D < 1 || E < 1) return 2;
+  return 0;
+}
+
+static void set_threads(int nthreads) {
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+}
+
+/* Masked sum: the definition, term by term. */
+int la_oracle_masked(const void* q, const void* k, const void* v, int dtype,
+                     const float* slopes, double* out,
+                     int64_t B, int64_t H, int64_t N, int64_t D, int64_t E, int nthreads) {
+  int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
+  if (rc) return rc;
+  set_threads(nthreads);
+  int64_t BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    double lam = (double)slopes[bh % H];
+    double* Q = (double*)malloc(sizeof(double) * (size_t)(N * D + 1));
+    double* K = (double*)malloc(sizeof(double) * (size_t)(N * D + 1));
+    double* V = (double*)malloc(sizeof(double) * (size_t)(N * E + 1));
+    in_row(Q, q, bh * N * D, N * D, dtype);
+    in_row(K, k, bh * N * D, N * D, dtype);
+    in_row(V, v, bh * N * E, N * E, dtype);
+    double* O = out + bh * N * E;
+    for (int64_t t = 0; t < N; ++t) {
+      for (int64_t e = 0; e < E; ++e) O[t * E + e] = 0.0;
+      for (int64_t s = 0; s <= t; ++s) {
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += Q[t * D + d] * K[s * D + d];
+        double w = exp(-lam * (double)(t - s)) * dot;
+        for (int64_t e = 0; e < E; ++e) O[t * E + e] += w * V[s * E + e];
+      }
+    }
+    free(Q);
+    free(K);
+    free(V);
+  }
+  return 0;
+}
+
+/*
+ * Recurrence S_t = gamma S_{t-1} + k_t^T v_t (S is D x E, row d, column e),
+ * o_t = q_t S_t.  s0 (nullable, [B][H][D][E]) is S_{-1}; zero if NULL.
+ * s_final (nullable) receives S_{N-1} (or s0 when N == 0).
+ */
+int la_oracle_recurrent(const void* q, const void* k, const void* v, int dtype,
+                        const float* slopes, const double* s0, double* s_final, double* out,
+                        int64_t B, int64_t H, int64_t N, int64_t D, int64_t E, int nthreads) {
+  int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
+  if (rc) return rc;
+  set_threads(nthreads);
+  int64_t BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    double gamma = exp(-(double)slopes[bh % H]);
+    double* S = (double*)calloc((size_t)(D * E), sizeof(double));
+    double* qt = (double*)malloc(sizeof(double) * (size_t)D);
+    double* kt = (double*)malloc(sizeof(double) * (size_t)D);
+    double* vt = (double*)malloc(sizeof(double) * (size_t)E);
+    if (s0) memcpy(S, s0 + bh * D * E, sizeof(double) * (size_t)(D * E));
+    double* O = out + bh * N * E;
+    for (int64_t t = 0; t < N; ++t) {
+      in_row(qt, q, (bh * N + t) * D, D, dtype);
+      in_row(kt, k, (bh * N + t) * D, D, dtype);
+      in_row(vt, v, (bh * N + t) * E, E, dtype);
+      for (int64_t d = 0; d < D; ++d)
+        for (int64_t e = 0; e < E; ++e) S[d * E + e] = gamma * S[d * E + e] + kt[d] * vt[e];
+      for (int64_t e = 0; e < E; ++e) O[t * E + e] = 0.0;
+      for (int64_t d = 0; d < D; ++d)
+        for (int64_t e = 0; e < E; ++e) O[t * E + e] += qt[d] * S[d * E + e];
+    }
+    if (s_final) memcpy(s_final + bh * D * E, S, sizeof(double) * (size_t)(D * E));
+    free(S);
+    free(qt);
+    free(kt);
+    free(vt);
+  }
+  return 0;
+}
+
+/*
+ * The recurrence, writing o_t only for t in pos[0..npos) (each 0 <= pos < N,
+ * any order) into out[B][H][npos][E].  Same arithmetic as la_oracle_recurrent.
+ */
+int la_oracle_recurrent_sampled(const void* q, const void* k, const void* v, int dtype,
+                                const float* slopes, const int64_t* pos, int64_t npos,
+                                double* out, int64_t B, int64_t H, int64_t N, int64_t D,
+                                int64_t E, int nthreads) {
+  int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
+  if (rc) return rc;
+  if (npos < 0 || (npos > 0 && !pos)) return 1;
+  for (int64_t p = 0; p < npos; ++p)
+    if (pos[p] < 0 || pos[p] >= N) return 2;
+  set_threads(nthreads);
+  int64_t BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    double gamma = exp(-(double)slopes[bh % H]);
+    double* S = (double*)calloc((size_t)(D * E), sizeof(double));
+    double* qt = (double*)malloc(sizeof(double) * (size_t)D);
+    double* kt = (double*)malloc(sizeof(double) * (size_t)D);
+    double* vt = (double*)malloc(sizeof(double) * (size_t)E);
+    unsigned char* want = (unsigned char*)calloc((size_t)(N + 1), 1);
+    for (int64_t p = 0; p < npos; ++p) want[pos[p]] = 1;
+    double* O = out + bh * npos * E;
+    for (int64_t t = 0; t < N; ++t) {
+      in_row(kt, k, (bh * N + t) * D, D, dtype);
+      in_row(vt, v, (bh * N + t) * E, E, dtype);
+      for (int64_t d = 0; d < D; ++d)
+        for (int64_t e = 0; e < E; ++e) S[d * E + e] = gamma * S[d * E + e] + kt[d] * vt[e];
+      if (!want[t]) continue;
+      in_row(qt, q, (bh * N + t) * D, D, dtype);
+      for (int64_t p = 0; p < npos; ++p) {
+        if (pos[p] != t) continue;
+        for (int64_t e = 0; e < E; ++e) {
+          double acc = 0.0;
+          for (int64_t d = 0; d < D; ++d) acc += qt[d] * S[d * E + e];
+          O[p * E + e] = acc;
+        }
+      }
+    }
+    free(S);
+    free(qt);
+    free(kt);
+    free(vt);
+    free(want);
+  }
+  return 0;
+}
+
+/*
+ * Blocked form with block size blk >= 1.  For the block [t0, t0 + len):
+ *   intra:  o_i += sum_{j <= i in block} exp(-lambda (i - j)) (q_i . k_j) v_j
+ *   inter:  o_i += exp(-lambda (i - t0 + 1)) q_i S_prev
+ *   carry:  S <- exp(-lambda len) S_prev + sum_j exp(-lambda (t0 + len - 1 - j)) k_j^T v_j
+ * Mathematically equal to the masked sum for every blk (blk = 1 is the
+ * recurrence, blk >= N the masked sum); only rounding differs.
+ */
+int la_oracle_blocked(const void* q, const void* k, const void* v, int dtype,
+                      const float* slopes, int64_t blk, double* out,
+                      int64_t B, int64_t H, int64_t N, int64_t D, int64_t E, int nthreads) {
+  int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
+  if (rc) return rc;
+  if (blk < 1) return 2;
+  set_threads(nthreads);
+  int64_t BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    double lam = (double)slopes[bh % H];
+    double* S = (double*)calloc((size_t)(D * E), sizeof(double));
+    double* Snew = (double*)malloc(sizeof(double) * (size_t)(D * E));
+    double* Q = (double*)malloc(sizeof(double) * (size_t)(blk * D));
+    double* K = (double*)malloc(sizeof(double) * (size_t)(blk * D));
+    double* V = (double*)malloc(sizeof(double) * (size_t)(blk * E));
+    double* O = out + bh * N * E;
+    for (int64_t t0 = 0; t0 < N; t0 += blk) {
+      int64_t len = (N - t0 < blk) ? (N - t0) : blk;
+      in_row(Q, q, (bh * N + t0) * D, len * D, dtype);
+      in_row(K, k, (bh * N + t0) * D, len * D, dtype);
+      in_row(V, v, (bh * N + t0) * E, len * E, dtype);
+      for (int64_t i = 0; i < len; ++i) {
+        double* o = O + (t0 + i) * E;
+        double a = exp(-lam * (double)(i + 1));
+        for (int64_t e = 0; e < E; ++e) {
+          double acc = 0.0;
+          for (int64_t d = 0; d < D; ++d) acc += Q[i * D + d] * S[d * E + e];
+          o[e] = a * acc;
+        }
+        for (int64_t j = 0; j <= i; ++j) {
+          double dot = 0.0;
+          for (int64_t d = 0; d < D; ++d) dot += Q[i * D + d] * K[j * D + d];
+          double p = exp(-lam * (double)(i - j)) * dot;
+          for (int64_t e = 0; e < E; ++e) o[e] += p * V[j * E + e];
+        }
+      }
+      double decay = exp(-lam * (double)len);
+      for (int64_t d = 0; d < D; ++d)
+        for (int64_t e = 0; e < E; ++e) Snew[d * E + e] = decay * S[d * E + e];
+      for (int64_t j = 0; j < len; ++j) {
+        double w = exp(-lam * (double)(len - 1 - j));
+        for (int64_t d = 0; d < D; ++d)
+          for (int64_t e = 0; e < E; ++e) Snew[d * E + e] += w * K[j * D + d] * V[j * E + e];
+      }
+      double* tmp = S;
+      S = Snew;
+      Snew = tmp;
+    }
+    free(S);
+    free(Snew);
+    free(Q);
+    free(K);
+    free(V);
+  }
+  return 0;
+}
+
+/*
+ * One recurrent decode step on state [B][H][D][E] (double, in place):
+ *   state <- exp(-lambda_h) state + k^T v ;  out = q . state (updated state).
+ * q, k are [B][H][D], v is [B][H][E], out is [B][H][E].
+ */
+int la_oracle_decode_step(const void* q, const void* k, const void* v, int dtype,
+                          const float* slopes, double* state, double* out,
+                          int64_t B, int64_t H, int64_t D, int64_t E, int nthreads) {
+  int rc = bad_args(q, k, v, slopes, out, B, H, 1, D, E);
+  if (rc) return rc;
+  if (!state) return 1;
+  set_threads(nthreads);
+  int64_t BH = B * H;
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    double gamma = exp(-(double)slopes[bh % H]);
+    double* S = state + bh * D * E;
+    double* o = out + bh * E;
+    for (int64_t d = 0; d < D; ++d) {
+      double kd = in_at(k, bh * D + d, dtype);
+      for (int64_t e = 0; e < E; ++e) S[d * E + e] = gamma * S[d * E + e] + kd * in_at(v, bh * E + e, dtype);
+    }
+    for (int64_t e = 0; e < E; ++e) o[e] = 0.0;
+    for (int64_t d = 0; d < D; ++d) {
+      double qd = in_at(q, bh * D + d, dtype);
+      for (int64_t e = 0; e < E; ++e) o[e] += qd * S[d * E + e];
+    }
+  }
+  return 0;
+}
+
+/* Number of threads an OpenMP parallel region would use (1 without OpenMP). */
+int la_oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
