@@ -75,6 +75,25 @@ int lightning_attn_fwd(const void* q, const void* k, const void* v,
                        int B, int H, int N, int D, int E, void* stream);
 
 /*
+ * lightning_attn_fwd with an optional initial state, an optional final state
+ * and an explicit chunk length.
+ *   init_state : nullable fp32 [B][H][D][E]; the state before token 0 (zero if
+ *                NULL).  Output rows then include exp(-lambda (t+1)) q_t S_0.
+ *   final_state: nullable fp32 [B][H][D][E]; receives the state after token
+ *                N-1, so a later call (or lightning_attn_decode) can continue
+ *                the sequence.
+ *   chunk      : tokens per chunk of the parallel sequence split, a multiple
+ *                of 128 (LA_ERR_SHAPE otherwise); 0 picks one from B*H, N and
+ *                the SM count.  The result does not depend on it beyond
+ *                rounding.
+ * Same layouts, alignment and errors as lightning_attn_fwd.
+ */
+int lightning_attn_fwd_ex(const void* q, const void* k, const void* v,
+                          const float* slopes, const float* init_state,
+                          float* final_state, float* out, int B, int H, int N,
+                          int D, int E, int chunk, void* stream);
+
+/*
  * Prefill with fp32 inputs and output (same operation and layout as
  * lightning_attn_fwd, all tensors fp32).  D, E in {64, 128}.  CUDA-core fp32
  * arithmetic, for callers that need fp32-class accuracy.

@@ -1,0 +1,231 @@
+// lightning_attn.cu -- C ABI of the library: argument checks, TMA tensor maps,
+// scratch for the chunked scan, and kernel launches.  Every compute step runs
+// in the kernels included below; the host code only marshals and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lightning_attn.h"
+#include "sm100_ptx.cuh"
+#include "tmap.h"
+
+namespace la {
+// Sticky device-side status word: bit 0 = an mbarrier wait ran out of time,
+// bit 1 = a chunk-scan flag wait ran out of time.
+__device__ int g_status;
+}  // namespace la
+
+#include "la_decode.cuh"
+#include "la_fwd_f32.cuh"
+#include "la_fwd_sm100.cuh"
+
+namespace {
+
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per device-side wait
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+inline bool dims_ok(int B, int H, int N, int D, int E) {
+  if (B < 1 || H < 1 || N < 1) return false;
+  const __int128 n = static_cast<__int128>(B) * H * N * (D > E ? D : E);
+  return n < (static_cast<__int128>(1) << 62) && static_cast<long long>(B) * H < (1ll << 31);
+}
+
+inline int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+inline int* status_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, la::g_status) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+    return 148;
+  return n;
+}
+
+// Chunk length for the sequence split: whole sequences when there are enough
+// of them, else chunks of at most 1024 tokens (their K/V stay in L2 between the
+// two phases) so that the work items cover several waves of SMs.
+int auto_chunk(int nseq, int N, int sms) {
+  const int nblk = (N + 127) / 128;
+  if (nseq >= 4 * sms || nblk <= 4) return nblk * 128;
+  const int want_chunks = (4 * sms + nseq - 1) / nseq;
+  int L = ((N + want_chunks - 1) / want_chunks + 127) / 128 * 128;
+  if (L < 512) L = 512;
+  if (L > 1024) L = 1024;
+  return L;
+}
+
+int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slopes,
+                  const float* init_state, float* final_state, float* out, int B, int H, int N,
+                  int D, int E, int chunk, void* stream_ptr) {
+  if (!q || !k || !v || !slopes || !out) return LA_ERR_NULL;
+  if (!dims_ok(B, H, N, D, E)) return LA_ERR_SHAPE;
+  if (D != 128 || E != 128) return LA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(slopes) ||
+      (init_state && !aligned16(init_state)) || (final_state && !aligned16(final_state)))
+    return LA_ERR_ALIGN;
+  if (chunk < 0 || (chunk % 128) != 0) return LA_ERR_SHAPE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  const int nseq = B * H;
+  const int sms = sm_count();
+  const int nblk = (N + 127) / 128;
+  int L = chunk > 0 ? chunk : auto_chunk(nseq, N, sms);
+  if (L >= nblk * 128) L = nblk * 128;
+  const int nchunks = (N + L - 1) / L;
+  const long long total = static_cast<long long>(nseq) * nchunks;
+  if (total >= (1ll << 31)) return LA_ERR_SHAPE;
+
+  CUtensorMap tq, tk, tv, to;
+  if (!la::make_tmap_3d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
+      !la::make_tmap_3d(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
+      !la::make_tmap_3d(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
+      !la::make_tmap_3d(&to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, N, nseq, 32, 128))
+    return LA_ERR_CUDA;
+
+  la::fwd::Params p{};
+  p.slopes = slopes;
+  p.init_state = init_state;
+  p.final_state = final_state;
+  p.status = status_word();
+  if (!p.status) return LA_ERR_CUDA;
+  p.H = H;
+  p.N = N;
+  p.nseq = nseq;
+  p.L = L;
+  p.nchunks = nchunks;
+  p.total = static_cast<int>(total);
+  p.wait_limit_ns = kWaitLimitNs;
+
+  void* scratch = nullptr;
+  if (nchunks > 1) {
+    const size_t ctrl = ((static_cast<size_t>(nseq) * 2 + 1) * sizeof(int) + 255) / 256 * 256;
+    const size_t bytes = ctrl + static_cast<size_t>(nseq) * 2 * 128 * 128 * sizeof(float);
+    if (cudaMallocAsync(&scratch, bytes, stream) != cudaSuccess) return LA_ERR_CUDA;
+    if (cudaMemsetAsync(scratch, 0, ctrl, stream) != cudaSuccess) {
+      cudaFreeAsync(scratch, stream);
+      return LA_ERR_CUDA;
+    }
+    p.ticket = static_cast<int*>(scratch);
+    p.flags = p.ticket + 1;
+    p.prefix = reinterpret_cast<float*>(static_cast<char*>(scratch) + ctrl);
+  }
+
+  // set on every call: the attribute belongs to the current device's context
+  const bool attr_ok =
+      cudaFuncSetAttribute(la::fwd::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           la::fwd::SMEM_BYTES) == cudaSuccess;
+  int rc = LA_OK;
+  if (!attr_ok) {
+    rc = LA_ERR_CUDA;
+  } else {
+    const int grid = static_cast<int>(total < sms ? total : sms);
+    la::fwd::fwd_bf16_kernel<<<grid, la::fwd::THREADS, la::fwd::SMEM_BYTES, stream>>>(tq, tk, tv,
+                                                                                    to, p);
+    rc = launch_status();
+  }
+  if (scratch && cudaFreeAsync(scratch, stream) != cudaSuccess) rc = LA_ERR_CUDA;
+  return rc;
+}
+
+template <int D, int E>
+int launch_f32(const float* q, const float* k, const float* v, const float* slopes, float* out,
+               int B, int H, int N, cudaStream_t stream) {
+  constexpr size_t smem = la::fwd_f32_smem_bytes<D, E>();
+  const bool attr_ok =
+      cudaFuncSetAttribute(la::fwd_f32_kernel<D, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) == cudaSuccess;
+  if (!attr_ok) return LA_ERR_CUDA;
+  la::fwd_f32_kernel<D, E><<<B * H, 256, smem, stream>>>(q, k, v, slopes, out, H, N);
+  return launch_status();
+}
+
+template <int D, int E>
+int launch_decode(const void* q, const void* k, const void* v, float* state, const float* slopes,
+                  float* out, int B, int H, cudaStream_t stream) {
+  la::decode_kernel<D, E><<<B * H, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), state, slopes, out, H);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int lightning_attn_fwd(const void* q, const void* k, const void* v, const float* slopes,
+                       float* out, int B, int H, int N, int D, int E, void* stream) {
+  return fwd_bf16_impl(q, k, v, slopes, nullptr, nullptr, out, B, H, N, D, E, 0, stream);
+}
+
+int lightning_attn_fwd_ex(const void* q, const void* k, const void* v, const float* slopes,
+                          const float* init_state, float* final_state, float* out, int B, int H,
+                          int N, int D, int E, int chunk, void* stream) {
+  return fwd_bf16_impl(q, k, v, slopes, init_state, final_state, out, B, H, N, D, E, chunk,
+                       stream);
+}
+
+int lightning_attn_fwd_f32(const float* q, const float* k, const float* v, const float* slopes,
+                           float* out, int B, int H, int N, int D, int E, void* stream) {
+  if (!q || !k || !v || !slopes || !out) return LA_ERR_NULL;
+  if (!dims_ok(B, H, N, D, E)) return LA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(slopes))
+    return LA_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (D == 64 && E == 64) return launch_f32<64, 64>(q, k, v, slopes, out, B, H, N, s);
+  if (D == 64 && E == 128) return launch_f32<64, 128>(q, k, v, slopes, out, B, H, N, s);
+  if (D == 128 && E == 64) return launch_f32<128, 64>(q, k, v, slopes, out, B, H, N, s);
+  if (D == 128 && E == 128) return launch_f32<128, 128>(q, k, v, slopes, out, B, H, N, s);
+  return LA_ERR_UNSUPPORTED;
+}
+
+int lightning_attn_decode(const void* q, const void* k, const void* v, float* state,
+                          const float* slopes, float* out, int B, int H, int D, int E,
+                          void* stream) {
+  if (!q || !k || !v || !state || !slopes || !out) return LA_ERR_NULL;
+  if (!dims_ok(B, H, 1, D, E)) return LA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) ||
+      !aligned16(out) || !aligned4(slopes))
+    return LA_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (D == 64 && E == 64) return launch_decode<64, 64>(q, k, v, state, slopes, out, B, H, s);
+  if (D == 64 && E == 128) return launch_decode<64, 128>(q, k, v, state, slopes, out, B, H, s);
+  if (D == 128 && E == 64) return launch_decode<128, 64>(q, k, v, state, slopes, out, B, H, s);
+  if (D == 128 && E == 128) return launch_decode<128, 128>(q, k, v, state, slopes, out, B, H, s);
+  return LA_ERR_UNSUPPORTED;
+}
+
+const char* lightning_attn_status_string(int status) {
+  switch (status) {
+    case LA_OK: return "LA_OK";
+    case LA_ERR_NULL: return "LA_ERR_NULL: a required pointer is NULL";
+    case LA_ERR_SHAPE: return "LA_ERR_SHAPE: invalid sizes";
+    case LA_ERR_ALIGN: return "LA_ERR_ALIGN: a tensor pointer is not 16-byte aligned";
+    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: unsupported head geometry";
+    case LA_ERR_CUDA: return "LA_ERR_CUDA: a CUDA call or kernel launch failed";
+    case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT: a device-side wait ran out of time";
+    case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE: workspace missing or too small";
+    default: return "unknown lightning_attn status";
+  }
+}
+
+int lightning_attn_device_status(int* status, int reset) {
+  if (!status) return LA_ERR_NULL;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, la::g_status, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
+  *status = v ? LA_ERR_TIMEOUT : LA_OK;
+  if (reset) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(la::g_status, &zero, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
+  }
+  return LA_OK;
+}
+
+}  // extern "C"

@@ -167,11 +167,19 @@ def decode_state(w: Workload) -> np.ndarray:
     return s
 
 
-def decode_step_inputs(w: Workload, step: int):
-    """q, k [B, H, D] and v [B, H, E] for one decode step, as bf16 bits."""
+def decode_step_inputs(w: Workload, step: int, rows: Optional[Sequence[int]] = None):
+    """q, k [B, H, D] and v [B, H, E] for one decode step, as bf16 bits.
+
+    Each batch row b has its own stream (keyed by tensor, b and step); rows
+    lists the batch rows to draw (others are zero), None draws all.
+    """
     out = []
+    todo = range(w.B) if rows is None else rows
     for name, width in (("q", w.D), ("k", w.D), ("v", w.E)):
-        x = _rng(w, name, 0, 0, step=step).standard_normal((w.B, w.H, width), dtype=np.float32)
+        x = np.zeros((w.B, w.H, width), np.float32)
+        for b in todo:
+            x[b] = _rng(w, name, b, 0, step=step + 1).standard_normal((w.H, width),
+                                                                      dtype=np.float32)
         x = _silu_f32(x) if name in ("q", "k") else x
         out.append(f32_to_bf16_bits(x))
     return tuple(out)

@@ -1,0 +1,166 @@
+"""Python binding of the C ABI in include/lightning_attn.h (argument marshalling only).
+
+Every function here checks tensor dtypes/shapes/devices, then calls the
+matching ``extern "C"`` entry point of ``liblightning_attn.so`` through ctypes
+on the current CUDA stream.  There is no other implementation behind these
+functions: if the library is missing or a call fails, they raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_SO = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblightning_attn.so")
+_lock = threading.Lock()
+_lib = None
+
+LA_OK = 0
+STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_NULL", 2: "LA_ERR_SHAPE", 3: "LA_ERR_ALIGN",
+                4: "LA_ERR_UNSUPPORTED", 5: "LA_ERR_CUDA", 6: "LA_ERR_TIMEOUT",
+                7: "LA_ERR_WORKSPACE"}
+
+# Exported entry points and their ctypes signatures (all return int).
+_P, _I = ctypes.c_void_p, ctypes.c_int
+SIGNATURES = {
+    "lightning_attn_fwd": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P],
+    "lightning_attn_fwd_ex": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P],
+    "lightning_attn_fwd_f32": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P],
+    "lightning_attn_decode": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P],
+    "lightning_attn_status_string": [_I],
+    "lightning_attn_device_status": [_P, _I],
+}
+
+
+class LightningAttnError(RuntimeError):
+    """A C-ABI call returned a non-zero status."""
+
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {status_string(code)} (code {code})")
+        self.code = code
+
+
+def library_path() -> str:
+    return _SO
+
+
+def lib():
+    """Loads liblightning_attn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_SO):
+                raise RuntimeError(
+                    f"{_SO} is missing: build it with `python -m long_context_fwd_b200.build` "
+                    "(or __graft_entry__.build()); there is no fallback implementation")
+            L = ctypes.CDLL(_SO)
+            for name, argtypes in SIGNATURES.items():
+                fn = getattr(L, name)
+                fn.argtypes = argtypes
+                fn.restype = ctypes.c_char_p if name == "lightning_attn_status_string" else _I
+            _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().lightning_attn_status_string(int(code)).decode()
+
+
+def _check(fn: str, rc: int):
+    if rc != LA_OK:
+        raise LightningAttnError(fn, rc)
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def fwd(q, k, v, slopes, out=None, *, init_state=None, final_state=None, chunk: int = 0,
+        stream=None) -> torch.Tensor:
+    """Prefill: bf16 q, k [B,H,N,D], v [B,H,N,E], fp32 slopes [H] -> fp32 out [B,H,N,E]."""
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    _need(q, "q", torch.bfloat16, (B, H, N, D))
+    _need(k, "k", torch.bfloat16, (B, H, N, D))
+    _need(v, "v", torch.bfloat16, (B, H, N, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    if out is None:
+        out = torch.empty((B, H, N, E), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, H, N, E))
+    for name, st in (("init_state", init_state), ("final_state", final_state)):
+        if st is not None:
+            _need(st, name, torch.float32, (B, H, D, E))
+    L = lib()
+    if init_state is None and final_state is None and chunk == 0:
+        rc = L.lightning_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), slopes.data_ptr(),
+                                  out.data_ptr(), B, H, N, D, E, _stream_handle(stream))
+        _check("lightning_attn_fwd", rc)
+    else:
+        rc = L.lightning_attn_fwd_ex(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), slopes.data_ptr(),
+            None if init_state is None else init_state.data_ptr(),
+            None if final_state is None else final_state.data_ptr(),
+            out.data_ptr(), B, H, N, D, E, int(chunk), _stream_handle(stream))
+        _check("lightning_attn_fwd_ex", rc)
+    return out
+
+
+def fwd_f32(q, k, v, slopes, out=None, *, stream=None) -> torch.Tensor:
+    """Prefill with fp32 q, k, v -> fp32 out."""
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    _need(q, "q", torch.float32, (B, H, N, D))
+    _need(k, "k", torch.float32, (B, H, N, D))
+    _need(v, "v", torch.float32, (B, H, N, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    if out is None:
+        out = torch.empty((B, H, N, E), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, H, N, E))
+    rc = lib().lightning_attn_fwd_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(), slopes.data_ptr(),
+                                      out.data_ptr(), B, H, N, D, E, _stream_handle(stream))
+    _check("lightning_attn_fwd_f32", rc)
+    return out
+
+
+def decode(q, k, v, state, slopes, out=None, *, stream=None) -> torch.Tensor:
+    """One decode step: bf16 q, k [B,H,D], v [B,H,E]; fp32 state [B,H,D,E] in place."""
+    B, H, D = q.shape
+    E = v.shape[-1]
+    _need(q, "q", torch.bfloat16, (B, H, D))
+    _need(k, "k", torch.bfloat16, (B, H, D))
+    _need(v, "v", torch.bfloat16, (B, H, E))
+    _need(state, "state", torch.float32, (B, H, D, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    if out is None:
+        out = torch.empty((B, H, E), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, H, E))
+    rc = lib().lightning_attn_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), state.data_ptr(),
+                                     slopes.data_ptr(), out.data_ptr(), B, H, D, E,
+                                     _stream_handle(stream))
+    _check("lightning_attn_decode", rc)
+    return out
+
+
+def device_status(reset: bool = True) -> int:
+    """Sticky device-side status of the current device (synchronises)."""
+    v = ctypes.c_int(0)
+    _check("lightning_attn_device_status",
+           lib().lightning_attn_device_status(ctypes.byref(v), 1 if reset else 0))
+    return v.value

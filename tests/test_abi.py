@@ -1,0 +1,96 @@
+"""The C-ABI library loads and exports every entry point of include/lightning_attn.h,
+and its host-side argument validation rejects bad calls before any launch (CPU only).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_fwd_b200 import build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lightning_attn.h")
+
+LA_ERR_NULL, LA_ERR_SHAPE, LA_ERR_ALIGN, LA_ERR_UNSUPPORTED = 1, 2, 3, 4
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(lightning_attn_\w+)\s*\(", text, flags=re.M)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ops.lib()
+
+
+def test_header_lists_entry_points():
+    names = header_functions()
+    assert "lightning_attn_fwd" in names and "lightning_attn_decode" in names
+    assert len(names) == len(set(names))
+
+
+def test_library_exports_every_header_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+        assert name in ops.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        s = ops.status_string(code)
+        assert s.startswith("LA_")
+    assert "unknown" in ops.status_string(99)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation first
+
+
+def test_fwd_validation(lib):
+    f = lib.lightning_attn_fwd
+    assert f(None, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 8, 128, 128, None) == LA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 128, 128, None) == LA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 128, 128, None) == LA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, -3, 8, 128, 128, None) == LA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 128, None) == LA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 128, 96, None) == LA_ERR_UNSUPPORTED
+    assert f(FAKE + 8, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_ALIGN
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE + 4, 1, 1, 8, 128, 128, None) == LA_ERR_ALIGN
+    assert f(FAKE, FAKE, FAKE, FAKE + 2, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_ALIGN
+    big = 1 << 30
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, big, big, big, 128, 128, None) == LA_ERR_SHAPE
+    g = lib.lightning_attn_fwd_ex
+    assert g(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 1, 8, 128, 128, 100, None) == LA_ERR_SHAPE
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE + 8, None, FAKE, 1, 1, 8, 128, 128, 0, None) == LA_ERR_ALIGN
+    assert g(FAKE, FAKE, FAKE, FAKE, None, FAKE + 8, FAKE, 1, 1, 8, 128, 128, 0, None) == LA_ERR_ALIGN
+
+
+def test_fwd_f32_validation(lib):
+    f = lib.lightning_attn_fwd_f32
+    assert f(FAKE, None, FAKE, FAKE, FAKE, 1, 1, 8, 64, 64, None) == LA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 64, 64, None) == LA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE + 4, FAKE, FAKE, 1, 1, 8, 64, 64, None) == LA_ERR_ALIGN
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 32, 64, None) == LA_ERR_UNSUPPORTED
+
+
+def test_decode_validation(lib):
+    f = lib.lightning_attn_decode
+    assert f(FAKE, FAKE, FAKE, None, FAKE, FAKE, 1, 1, 128, 128, None) == LA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 128, 128, None) == LA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE + 8, FAKE, FAKE, 1, 1, 128, 128, None) == LA_ERR_ALIGN
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 256, None) == LA_ERR_UNSUPPORTED
+
+
+def test_device_status_null(lib):
+    assert lib.lightning_attn_device_status(None, 0) == LA_ERR_NULL
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ops.fwd(x, x, x, torch.zeros(1))

@@ -1,0 +1,200 @@
+"""GPU parity of the prefill entry points against the float64 oracle.
+
+Every case calls the CUDA library through its C ABI (long_context_fwd_b200.ops)
+and compares element by element with the oracle on the same seeded inputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_fwd_b200 import inputs as I
+from long_context_fwd_b200 import ops
+from parity import TOL_BF16, TOL_F32, bf16_to_dev, f32_to_dev, rel, worst_head
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+def _bf16_case(B, H, N, slopes, seed):
+    w = I.Workload(f"case{seed}", B, H, N, 128, 128, "bf16", index=100 + seed)
+    q, k, v = I.prefill_inputs(w)
+    return q, k, v, np.asarray(slopes, np.float32)
+
+
+def _run(q, k, v, sl, **kw):
+    out = ops.fwd(bf16_to_dev(q, DEV), bf16_to_dev(k, DEV), bf16_to_dev(v, DEV),
+                  f32_to_dev(sl, DEV), **kw)
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("w", [I.TINY_F32, I.TINY_F32_NODECAY], ids=lambda w: w.name)
+def test_f32_tiny_workload(w):
+    q, k, v = I.prefill_inputs(w)
+    sl = I.slopes_for(w)
+    out = ops.fwd_f32(*(f32_to_dev(x, DEV) for x in (q, k, v)), f32_to_dev(sl, DEV))
+    got = out.cpu().numpy()
+    ref = oracle.masked(q, k, v, sl)
+    assert rel(got, ref) <= TOL_F32
+    assert worst_head(got, ref) <= TOL_F32
+    # block size 64 of the workload recipe: the blocked oracle agrees with the definition
+    assert rel(oracle.blocked(q, k, v, sl, 64), ref) <= 1e-12
+
+
+@pytest.mark.parametrize("D,E", [(64, 128), (128, 64), (128, 128)])
+def test_f32_other_head_geometries(D, E):
+    w = I.Workload("f32geo", 2, 2, 301, D, E, "f32", index=90)
+    q, k, v = I.prefill_inputs(w)
+    sl = np.array([0.3, 0.0], np.float32)
+    out = ops.fwd_f32(*(f32_to_dev(x, DEV) for x in (q, k, v)), f32_to_dev(sl, DEV))
+    assert rel(out.cpu().numpy(), oracle.recurrent(q, k, v, sl)) <= TOL_F32
+
+
+BF16_CASES = [
+    # B, H, N, slopes, chunk
+    (1, 1, 1, [0.5], 0),
+    (1, 1, 63, [0.3], 0),
+    (1, 1, 128, [0.1], 0),
+    (1, 2, 129, [0.0, 0.9], 0),
+    (1, 3, 257, [0.0, 0.05, 5.0], 0),
+    (2, 3, 777, [0.917, 0.25, 0.0], 0),
+    (1, 2, 1024, [0.2, 0.0], 256),
+    (1, 4, 3000, [0.9, 0.3, 0.0, 0.01], 512),
+    (3, 4, 2100, [0.9, 0.3, 0.0, 0.01], 128),
+    (1, 2, 4097, [0.004, 0.0], 1024),
+]
+
+
+@pytest.mark.parametrize("B,H,N,slopes,chunk", BF16_CASES)
+def test_bf16_parity_shapes(B, H, N, slopes, chunk):
+    q, k, v, sl = _bf16_case(B, H, N, slopes, seed=N % 97 + B)
+    got = _run(q, k, v, sl, chunk=chunk)
+    ref = oracle.recurrent(q, k, v, sl)
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+
+
+def test_bf16_chunk_length_does_not_change_result():
+    q, k, v, sl = _bf16_case(2, 2, 2500, [0.3, 0.0], seed=11)
+    ref = oracle.recurrent(q, k, v, sl)
+    outs = [_run(q, k, v, sl, chunk=c) for c in (0, 128, 384, 1024, 2560)]
+    for o in outs:
+        assert rel(o, ref) <= TOL_BF16
+    for o in outs[1:]:
+        assert rel(o, outs[0]) <= 5e-3
+
+
+def test_bf16_deterministic():
+    q, k, v, sl = _bf16_case(1, 3, 3000, [0.5, 0.05, 0.0], seed=12)
+    a = _run(q, k, v, sl, chunk=256)
+    b = _run(q, k, v, sl, chunk=256)
+    assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("chunk", [0, 256])
+def test_bf16_initial_and_final_state(chunk):
+    B, H, N = 1, 3, 1500
+    q, k, v, sl = _bf16_case(B, H, N, [0.4, 0.0, 0.02], seed=13)
+    s0 = (np.random.default_rng(5).standard_normal((B, H, 128, 128)) * 0.02).astype(np.float32)
+    fin = torch.zeros((B, H, 128, 128), dtype=torch.float32, device=DEV)
+    got = _run(q, k, v, sl, init_state=f32_to_dev(s0, DEV), final_state=fin, chunk=chunk)
+    ref, sref = oracle.recurrent(q, k, v, sl, s0=s0.astype(np.float64), return_state=True)
+    assert rel(got, ref) <= TOL_BF16
+    assert rel(fin.cpu().numpy(), sref) <= TOL_BF16
+
+
+def test_bf16_prefill_then_decode_continues_sequence():
+    B, H, N, T = 2, 2, 700, 6
+    w = I.Workload("handoff", B, H, N + T, 128, 128, "bf16", index=140)
+    q, k, v = I.prefill_inputs(w)
+    sl = np.array([0.3, 0.0], np.float32)
+    state = torch.zeros((B, H, 128, 128), dtype=torch.float32, device=DEV)
+    _run(q[:, :, :N], k[:, :, :N], v[:, :, :N], sl, final_state=state, chunk=256)
+    ref = oracle.recurrent(q, k, v, sl)
+    ts = f32_to_dev(sl, DEV)
+    for t in range(N, N + T):
+        o = ops.decode(bf16_to_dev(q[:, :, t], DEV), bf16_to_dev(k[:, :, t], DEV),
+                       bf16_to_dev(v[:, :, t], DEV), state, ts)
+        assert rel(o.cpu().numpy(), ref[:, :, t]) <= TOL_BF16
+
+
+def test_bf16_degenerate_inputs():
+    B, H, N = 1, 2, 300
+    z = np.zeros((B, H, N, 128), np.uint16)
+    got = _run(z, z, z, np.array([0.1, 0.0], np.float32))
+    assert np.all(got == 0.0)
+    # gamma -> 0: only the diagonal term survives
+    q, k, v, _ = _bf16_case(B, H, N, [0, 0], seed=14)
+    sl = np.array([40.0, 60.0], np.float32)
+    got = _run(q, k, v, sl, chunk=128)
+    Q, K, V = (I.bf16_bits_to_f32(x).astype(np.float64) for x in (q, k, v))
+    diag = np.sum(Q * K, axis=-1, keepdims=True) * V
+    assert rel(got, diag) <= TOL_BF16
+
+
+def test_bf16_prefill_8k_workload_full():
+    """The B=1, H=64, N=8192 workload, every output element against the oracle."""
+    w = I.PREFILL_8K
+    q, k, v = I.prefill_inputs(w)
+    sl = I.slopes_for(w)
+    got = _run(q, k, v, sl)
+    ref = oracle.recurrent(q, k, v, sl)
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+
+
+def _device_workload_with_host_heads(w, heads):
+    """Full-size inputs on the device (torch generator) with the listed heads
+    replaced by the host generator's draws, which the oracle also consumes."""
+    q, k, v = I.device_prefill_inputs(w, DEV)
+    host = {}
+    for b, h in heads:
+        hq, hk, hv = I.head_inputs(w, b, h)
+        q[b, h].copy_(bf16_to_dev(hq, DEV))
+        k[b, h].copy_(bf16_to_dev(hk, DEV))
+        v[b, h].copy_(bf16_to_dev(hv, DEV))
+        host[(b, h)] = (hq, hk, hv)
+    return q, k, v, host
+
+
+def test_bf16_prefill_32k_workload_sampled_heads():
+    """B=4, H=64, N=32768 (lambda = 0 on heads h % 8 == 7), as the benchmark runs
+    it; eight heads (three with lambda = 0) compared in full against the oracle."""
+    w = I.PREFILL_32K
+    heads = [(0, 0), (0, 7), (1, 31), (1, 63), (2, 15), (2, 40), (3, 1), (3, 55)]
+    sl = I.slopes_for(w)
+    q, k, v, host = _device_workload_with_host_heads(w, heads)
+    out = ops.fwd(q, k, v, f32_to_dev(sl, DEV))
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0
+    del q, k, v
+    for (b, h), (hq, hk, hv) in host.items():
+        ref = oracle.recurrent(hq[None, None], hk[None, None], hv[None, None], sl[h:h + 1])
+        got = out[b, h].cpu().numpy()
+        assert rel(got, ref[0, 0]) <= TOL_BF16, (b, h)
+    assert torch.isfinite(out).all()
+
+
+@pytest.mark.slow
+def test_bf16_prefill_1m_workload_sampled():
+    """B=1, H=64, N=1,048,576: three heads checked at 64 sampled positions each
+    against the oracle's recurrence."""
+    w = I.PREFILL_1M
+    heads = [(0, 0), (0, 31), (0, 63)]
+    sl = I.slopes_for(w)
+    q, k, v, host = _device_workload_with_host_heads(w, heads)
+    out = ops.fwd(q, k, v, f32_to_dev(sl, DEV))
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0
+    del q, k, v
+    pos = I.sample_positions(w.N)
+    hq = np.stack([host[x][0] for x in heads])[None]
+    hk = np.stack([host[x][1] for x in heads])[None]
+    hv = np.stack([host[x][2] for x in heads])[None]
+    ref = oracle.recurrent_sampled(hq, hk, hv, sl[[h for _, h in heads]], pos)
+    idx = torch.as_tensor(pos, device=DEV)
+    for i, (b, h) in enumerate(heads):
+        got = out[b, h].index_select(0, idx).cpu().numpy()
+        assert rel(got, ref[0, i]) <= TOL_BF16, (b, h)
