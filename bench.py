@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the Lightning Attention hot path on B200 (one JSON line on rank 0).
+
+Default workload (the prefill configuration the throughput target is stated
+for, N >= 32K): B=4, H=64, N=32768, D=E=128, bf16 q/k/v, fp32 out, ALiBi-style
+slopes with lambda = 0 on heads h % 8 == 7.  A step is one lightning_attn_fwd
+call over the whole batch (q, k, v resident in HBM, 10.7 GB moved per step --
+larger than L2, so no flush is needed).  The same line carries the decode leg
+(256 sequences x 64 heads, fp32 128x128 states, 1024 chained
+lightning_attn_decode steps), the end-to-end number through host buffers, the
+roofline of the prefill kernel and the float64 oracle timed on the host cores.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs the full workload on
+its own GPU -- independent (b, h) problems, no collective on the data path --
+and the reported throughput is the whole job's tokens over the slowest rank's
+device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "lightning-attn prefill tokens/s (% roofline); decode tokens/s (HBM GB/s)"
+BYTES_PER_TOKEN_HEAD = 2 * 128 + 2 * 128 + 2 * 128 + 4 * 128  # q, k, v bf16 in + out fp32
+BLK = 128  # tokens per block in the prefill kernel
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_b4h64n32768d128")
+    ap.add_argument("--chunk", type=int, default=0, help="prefill chunk length (0 = automatic)")
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-decode", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(device_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        self.windows = []
+
+    def mark(self, t0: float, t1: float):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                    rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
+                except Exception:
+                    continue
+        os.unlink(self.tmp.name)
+        inside = [r for r in rows if any(a - 0.05 <= r[0] <= b + 0.05 for a, b in self.windows)]
+        use = inside if inside else rows[-5:]
+        if not use:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use), "in_timed_region": bool(inside)}
+
+
+# ----------------------------------------------------------------------------
+# our implementation
+# ----------------------------------------------------------------------------
+def bench_prefill(args, dist, w, dev):
+    import torch
+    from long_context_fwd_b200 import inputs as I
+    from long_context_fwd_b200 import ops
+
+    q, k, v = I.device_prefill_inputs(w, dev)
+    sl = torch.from_numpy(I.slopes_for(w)).to(dev)
+    out = torch.empty((w.B, w.H, w.N, w.E), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        ops.fwd(q, k, v, sl, out, chunk=args.chunk)
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0, "device-side wait timed out during warm-up"
+    dist.barrier()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_host0 = time.time()
+    for i in range(args.steps):
+        starts[i].record(stream)
+        ops.fwd(q, k, v, sl, out, chunk=args.chunk)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.time()
+    dist.barrier()
+    total_ms = starts[0].elapsed_time(ends[-1])
+    launch_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    status = ops.device_status(reset=True)
+    res = {"total_ms": dist.max(total_ms), "launch_ms": dist.max(launch_ms),
+           "window": (t_host0, t_host1), "status": status}
+    # end to end through host buffers: pinned inputs in, result out, every step
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    del q, k, v
+    torch.cuda.empty_cache()
+    dq, dk, dv = (torch.empty(x.shape, dtype=x.dtype, device=dev) for x in (hq, hk, hv))
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        ops.fwd(dq, dk, dv, sl, out, chunk=args.chunk)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    res["e2e_ms"] = dist.max(e0.elapsed_time(e1)) / args.e2e_steps
+    res["h2d"] = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    res["d2h"] = hout.numel() * hout.element_size()
+    del dq, dk, dv, hq, hk, hv, hout, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_decode(args, dist, dev):
+    import torch
+    from long_context_fwd_b200 import inputs as I
+    from long_context_fwd_b200 import ops
+
+    w = I.DECODE
+    steps = args.decode_steps
+    g = torch.Generator(device=dev)
+    g.manual_seed(4321)
+    state = torch.randn((w.B, w.H, w.D, w.E), generator=g, device=dev) * 0.02
+    sl = torch.from_numpy(I.slopes_for(w)).to(dev)
+    qs = torch.nn.functional.silu(torch.randn((steps, w.B, w.H, w.D), generator=g, device=dev)).to(torch.bfloat16)
+    ks = torch.nn.functional.silu(torch.randn((steps, w.B, w.H, w.D), generator=g, device=dev)).to(torch.bfloat16)
+    vs = torch.randn((steps, w.B, w.H, w.E), generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty((w.B, w.H, w.E), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for i in range(max(3, args.warmup)):
+        ops.decode(qs[i % steps], ks[i % steps], vs[i % steps], state, sl, out)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_host0 = time.time()
+    e0.record(stream)
+    for i in range(steps):
+        ops.decode(qs[i], ks[i], vs[i], state, sl, out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.time()
+    dist.barrier()
+    ms = dist.max(e0.elapsed_time(e1)) / steps
+    bytes_step = w.B * w.H * (2 * w.D * w.E * 4 + 2 * w.D * 2 + 2 * w.E + 4 * w.E + 4)
+    finite = bool(torch.isfinite(state).all().item())
+    del qs, ks, vs, state
+    torch.cuda.empty_cache()
+    return {"ms": ms, "bytes": bytes_step, "steps": steps, "window": (t_host0, t_host1),
+            "finite": finite, "workload": w.name, "tokens": w.B}
+
+
+def cpu_baseline(w, seconds: float):
+    """The float64 oracle's recurrence on a bounded prefix of the workload:
+    batch row 0, all H heads, the first n tokens (n sized to ~`seconds`)."""
+    import numpy as np
+    import oracle
+    from long_context_fwd_b200 import inputs as I
+
+    sl = I.slopes_for(w)
+
+    def run(n):
+        arrs = [I.head_inputs(w, 0, h, 0, n) for h in range(w.H)]
+        q = np.stack([a[0] for a in arrs])[None]
+        k = np.stack([a[1] for a in arrs])[None]
+        v = np.stack([a[2] for a in arrs])[None]
+        t0 = time.time()
+        oracle.recurrent(q, k, v, sl)
+        return time.time() - t0
+
+    n = 128
+    dt = run(n)
+    n = int(min(w.N, max(n, n * seconds / max(dt, 1e-3) * 0.9)))
+    dt = run(n)
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"float64 recurrence, batch row 0, all {w.H} heads, first {n} of {w.N} tokens "
+                      f"({dt:.1f} s)"}
+
+
+def main_ours(args):
+    import torch
+    from long_context_fwd_b200 import inputs as I
+
+    dist = Dist()
+    torch.cuda.set_device(dist.local)
+    dev = torch.device("cuda", dist.local)
+    dist.init("nccl")
+    w = I.WORKLOADS[args.workload]
+    hbm, bf16, peak_src = peaks()
+    sampler = ClockSampler(dist.local)
+    pre = bench_prefill(args, dist, w, dev)
+    sampler.mark(*pre["window"])
+    dec = None if args.no_decode else bench_decode(args, dist, dev)
+    clocks = sampler.stop()
+    tokens_step = w.B * w.N
+    ms_step = pre["total_ms"] / args.steps
+    value = dist.world * tokens_step / (ms_step / 1e3)
+    bytes_launch = w.B * w.H * w.N * BYTES_PER_TOKEN_HEAD
+    achieved = bytes_launch / (pre["launch_ms"] / 1e3) / 1e9
+    flops_launch = w.B * w.H * w.N * (4 * w.D * w.E + 2 * BLK * (w.D + w.E))
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded torch generator on the device; q, k = SiLU(N(0,1)), v = N(0,1))",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "E": w.E,
+                   "global_batch": w.B * dist.world, "seq_len": w.N, "chunk": args.chunk or "auto",
+                   "parallelism": f"replicas x{dist.world} (independent (b,h) problems, no collective)",
+                   "l2": "no flush: each step streams 10.7 GB, far larger than the 126 MB L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "peak_source": f"{peak_src} copy bandwidth",
+                     "bytes_per_launch": bytes_launch, "kernel_ms": pre["launch_ms"],
+                     "tensor_tflops": flops_launch / (pre["launch_ms"] / 1e3) / 1e12,
+                     "tensor_peak_tflops": bf16},
+        "gpu_launches": args.steps,
+        "device_status": pre["status"],
+        "e2e": {"value": dist.world * tokens_step / (pre["e2e_ms"] / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"],
+                "ms_per_step": pre["e2e_ms"]},
+        "clocks": clocks,
+    }
+    if dec:
+        gbs = dec["bytes"] / (dec["ms"] / 1e3) / 1e9
+        line["decode"] = {"workload": dec["workload"], "value": dist.world * dec["tokens"] / (dec["ms"] / 1e3),
+                          "unit": "tokens/s", "ms_per_step": dec["ms"], "steps": dec["steps"],
+                          "gpu_launches": dec["steps"], "state_finite": dec["finite"],
+                          "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                                       "frac": gbs / hbm, "bytes_per_launch": dec["bytes"]}}
+    if dist.rank == 0 and dist.world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host cores
+# ----------------------------------------------------------------------------
+def main_reference(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import numpy as np
+    import oracle
+    from long_context_fwd_b200 import inputs as I
+
+    w = I.WORKLOADS[args.workload]
+    sl = I.slopes_for(w)
+    budget = 120.0  # seconds for the whole reference run
+    per_step = budget / max(1, args.steps + args.warmup)
+
+    def sample(n):
+        arrs = [I.head_inputs(w, 0, h, 0, n) for h in range(w.H)]
+        return (np.stack([a[i] for a in arrs])[None] for i in range(3))
+
+    q, k, v = sample(64)
+    t0 = time.time()
+    oracle.recurrent(q, k, v, sl)
+    rate = 64 / max(time.time() - t0, 1e-4)
+    n = int(min(w.N, max(64, rate * per_step)))
+    q, k, v = sample(n)
+    for _ in range(args.warmup):
+        oracle.recurrent(q, k, v, sl)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.time()
+        oracle.recurrent(q, k, v, sl)
+        times.append(time.time() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = n / (ms / 1e3)
+    sample_desc = (f"float64 recurrence, batch row 0, all {w.H} heads, first {n} of {w.N} tokens "
+                   f"per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy generator)",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "E": w.E},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(),
+                             "kind": "oracle", "sample": sample_desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        main_reference(a)
+    else:
+        main_ours(a)
