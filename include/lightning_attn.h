@@ -115,6 +115,12 @@ int lightning_attn_decode(const void* q, const void* k, const void* v,
                           float* state, const float* slopes, float* out,
                           int B, int H, int D, int E, void* stream);
 
+/*
+ * Text of the CUDA runtime error behind the calling thread's most recent
+ * LA_ERR_CUDA (static string, never NULL; "no error" before any).
+ */
+const char* lightning_attn_last_cuda_error(void);
+
 /* Human-readable name of a la_status value (static string, never NULL). */
 const char* lightning_attn_status_string(int status);
 

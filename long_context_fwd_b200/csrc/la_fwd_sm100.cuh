@@ -20,18 +20,27 @@
 // state A_c = sum_j gamma^(Lc-1-j) k_j^T v_j over its tokens (phase 1, K/V
 // kept in L2 with an evict-last hint), then takes the inclusive state of the
 // previous chunk from global memory (spin on a flag, bounded in time),
-// publishes its own inclusive state gamma^Lc S_prev + A_c, and finally runs
-// the blocked form from S_prev (phase 2, re-reading K/V from L2).  Items are
-// handed out through an atomic ticket, so every chunk's predecessor is held by
-// a CTA that is already running: no co-residency assumption.
+// publishes its own inclusive state gamma^Lc S_prev + A_c, and runs the
+// blocked form from S_prev (phase 2, re-reading K/V from L2).  Items are handed
+// out through an atomic ticket, so every chunk's predecessor is held by a CTA
+// that is already running: no co-residency assumption.
 //
-// Roles (320 threads, one CTA per SM):
-//   warp 8      TMA producer: Q/K/V tiles into three 2-slot rings.
-//   warp 9      TMEM allocator and single-thread tcgen05.mma issuer.
-//   warps 0..7  compute: mask/scale (P, gamma^(i+1) Q, decayed K), the state
-//               copy to bf16 and its decay, the chunk scan, and the epilogue
-//               (TMEM -> swizzled shared memory -> TMA store of fp32 out).
+// Roles (448 threads, one CTA per SM):
+//   warps 0..7   group X: decay-causal mask of Q K^T into P (bf16, TMEM),
+//                gamma^(i+1) Q into TMEM, decayed K in place in shared memory.
+//                Thread t owns TMEM lane / tile row r = 32 (warp % 4) + lane and
+//                the column half hf = warp / 4.
+//   warps 8..11  group Y: the state's bf16 copy and decay, the chunk scan, and
+//                the epilogue (TMEM -> swizzled shared memory -> TMA store).
+//                Thread t owns row r = 32 (warp % 4) + lane, all 128 columns.
+//   warp 12      TMA producer: Q/K/V tiles into three 2-slot rings.
+//   warp 13      TMEM allocator and single-thread tcgen05.mma issuer.
+// X and Y run concurrently on different blocks' data.
 // TMEM (512 columns): S/P double buffer [0,256), O [256,384), state [384,512).
+// After group X has read the scores of an S buffer it rewrites the buffer with
+// two bf16 operands for the MMAs that follow: P (columns j < 64 in [0,32), j >= 64
+// in [64,96)) and gamma^(i+1) Q (d < 64 in [32,64), d >= 64 in [96,128)).  Each
+// thread overwrites only columns it has read itself.
 #pragma once
 
 #include <cuda.h>
@@ -43,23 +52,25 @@
 namespace la {
 namespace fwd {
 
-constexpr int BLK = 128;   // tokens per block (= MMA M)
-constexpr int HD = 128;    // D = E = 128
-constexpr int C_WARPS = 8;
-constexpr int C_THREADS = 32 * C_WARPS;
-constexpr int PRODUCER_WARP = 8;
-constexpr int MMA_WARP = 9;
-constexpr int THREADS = 320;
+constexpr int BLK = 128;  // tokens per block (= MMA M)
+constexpr int HD = 128;   // D = E = 128
+constexpr int X_THREADS = 256;
+constexpr int Y_THREADS = 128;
+constexpr int X_WARP0 = 0;
+constexpr int Y_WARP0 = 8;
+constexpr int PRODUCER_WARP = 12;
+constexpr int MMA_WARP = 13;
+constexpr int THREADS = 448;
 
-constexpr uint32_t PLANE = 16384;             // 128 rows x 128 B
-constexpr uint32_t TILE = 2 * PLANE;          // 128 x 128 bf16
-constexpr uint32_t OFF_Q = 0;                 // 2 slots
-constexpr uint32_t OFF_K = 2 * TILE;          // 2 slots
-constexpr uint32_t OFF_V = 4 * TILE;          // 2 slots
-constexpr uint32_t OFF_KVB = 6 * TILE;        // bf16 copy of the state (MMA B operand)
+constexpr uint32_t PLANE = 16384;       // 128 rows x 128 B
+constexpr uint32_t TILE = 2 * PLANE;    // 128 x 128 bf16
+constexpr uint32_t OFF_Q = 0;           // 2 slots
+constexpr uint32_t OFF_K = 2 * TILE;    // 2 slots
+constexpr uint32_t OFF_V = 4 * TILE;    // 2 slots
+constexpr uint32_t OFF_KVB = 6 * TILE;  // bf16 copy of the state (MMA B operand)
 constexpr uint32_t OFF_BAR = 7 * TILE;
-constexpr uint32_t OFF_GPOW = OFF_BAR + 512;  // gamma^m, m = 0..128
-constexpr uint32_t OFF_MISC = OFF_GPOW + 544;
+constexpr uint32_t OFF_GTAB = OFF_BAR + 512;  // 256 floats: gtab[u] = gamma^(127-u), 0 for u > 127
+constexpr uint32_t OFF_MISC = OFF_GTAB + 1024;
 constexpr uint32_t SMEM_USED = OFF_MISC + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
@@ -70,9 +81,9 @@ enum BarId : int {
   B_SF = 12, B_SE = 14,
   B_READY = 16, B_KVB_READY, B_KVO_DONE, B_O_FULL, B_O_EMPTY, B_AGG_FULL, B_KV_FREE,
   B_WF = 24, B_WE = 26,
-  B_CSYNC = 28, B_DRAIN = 29,
-  B_KT = 30,  // phase 1: decayed K tile ready, one per K slot (2)
-  B_COUNT = 32
+  B_XSYNC = 28, B_YSYNC = 29, B_DRAIN = 30,
+  B_KT = 32,  // phase 1: decayed K tile ready, one per K slot (2)
+  B_COUNT = 34
 };
 
 struct Params {
@@ -84,6 +95,7 @@ struct Params {
   float* final_state;         // nullable [nseq][HD*HD]
   int* status;                // sticky error word
   int H, N, nseq, L, nchunks, total;
+  int ticket_base;            // first ticket handed out (0 except in fault-injection runs)
   unsigned long long wait_limit_ns;
 };
 
@@ -91,6 +103,20 @@ struct Item {
   int seq, chunk, t0, Lc, nb;
   bool phase1;
 };
+
+// Optional event trace (compiled only with -DLA_TRACE): %globaltimer stamps of
+// each role's pipeline events for the first few CTAs, for timeline analysis.
+#ifdef LA_TRACE
+constexpr int TRACE_CTAS = 4, TRACE_EVENTS = 24, TRACE_SLOTS = 256;
+__device__ unsigned long long* g_trace;
+__device__ __forceinline__ void trace_event(int ev, uint32_t idx) {
+  if (g_trace && blockIdx.x < TRACE_CTAS && idx < TRACE_SLOTS)
+    g_trace[(blockIdx.x * TRACE_EVENTS + ev) * TRACE_SLOTS + idx] = globaltimer_ns();
+}
+#define LA_TRACE_EVENT(ev, idx) trace_event((ev), (idx))
+#else
+#define LA_TRACE_EVENT(ev, idx) ((void)0)
+#endif
 
 __device__ __forceinline__ Item decode_item(const Params& p, int w) {
   Item it;
@@ -112,83 +138,103 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* ptr) {
   return v;
 }
 
-// Multiplies the 64 bf16 of one 128-byte swizzled row by f, in place.  The
-// physical chunk order (c ^ row) keeps 8 consecutive rows on distinct banks.
-__device__ __forceinline__ void scale_row(uint8_t* rowp, uint32_t row, float f) {
-#pragma unroll
-  for (uint32_t c = 0; c < 8; ++c) {
-    uint4* p = reinterpret_cast<uint4*>(rowp + ((c ^ (row & 7u)) << 4));
-    uint4 x = *p;
-    x.x = pack_bf16x2(bf16lo_to_f32(x.x) * f, bf16hi_to_f32(x.x) * f);
-    x.y = pack_bf16x2(bf16lo_to_f32(x.y) * f, bf16hi_to_f32(x.y) * f);
-    x.z = pack_bf16x2(bf16lo_to_f32(x.z) * f, bf16hi_to_f32(x.z) * f);
-    x.w = pack_bf16x2(bf16lo_to_f32(x.w) * f, bf16hi_to_f32(x.w) * f);
-    *p = x;
-  }
+// ---------------------------------------------------------------------------
+// Shared-memory access with explicit state-space instructions
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ float lds32f(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts32f(uint32_t a, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
 }
 
-// Writes 64 floats as bf16 into one 128-byte swizzled row (logical chunk c
-// holds elements 8c..8c+7).
-__device__ __forceinline__ void store_row_bf16(uint8_t* rowp, uint32_t row, const float* x) {
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t x, float f) {
+  return pack_bf16x2(bf16lo_to_f32(x) * f, bf16hi_to_f32(x) * f);
+}
+
+// Multiplies the 64 bf16 of one 128-byte swizzled row by f, in place.  All 8
+// loads are issued before any store; the physical chunk order (c ^ row) keeps
+// 8 consecutive rows on distinct banks.
+__device__ __forceinline__ void scale_row(uint32_t rowaddr, uint32_t row, float f) {
+  uint4 x[8];
+#pragma unroll
+  for (uint32_t c = 0; c < 8; ++c) x[c] = lds128(rowaddr + ((c ^ (row & 7u)) << 4));
 #pragma unroll
   for (uint32_t c = 0; c < 8; ++c) {
+    x[c].x = scale_bf16x2(x[c].x, f);
+    x[c].y = scale_bf16x2(x[c].y, f);
+    x[c].z = scale_bf16x2(x[c].z, f);
+    x[c].w = scale_bf16x2(x[c].w, f);
+  }
+#pragma unroll
+  for (uint32_t c = 0; c < 8; ++c) sts128(rowaddr + ((c ^ (row & 7u)) << 4), x[c]);
+}
+
+// Writes 32 floats (times f) as bf16 into logical chunks [4*h, 4*h+4) of a
+// 128-byte swizzled row (logical chunk c holds row elements 8c..8c+7).
+__device__ __forceinline__ void store_half_bf16(uint32_t rowaddr, uint32_t row, uint32_t h,
+                                                const uint32_t (&x)[32], float f) {
+#pragma unroll
+  for (uint32_t c = 0; c < 4; ++c) {
     uint4 u;
-    u.x = pack_bf16x2(x[8 * c + 0], x[8 * c + 1]);
-    u.y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
-    u.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
-    u.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
-    *reinterpret_cast<uint4*>(rowp + ((c ^ (row & 7u)) << 4)) = u;
+    u.x = pack_bf16x2(__uint_as_float(x[8 * c + 0]) * f, __uint_as_float(x[8 * c + 1]) * f);
+    u.y = pack_bf16x2(__uint_as_float(x[8 * c + 2]) * f, __uint_as_float(x[8 * c + 3]) * f);
+    u.z = pack_bf16x2(__uint_as_float(x[8 * c + 4]) * f, __uint_as_float(x[8 * c + 5]) * f);
+    u.w = pack_bf16x2(__uint_as_float(x[8 * c + 6]) * f, __uint_as_float(x[8 * c + 7]) * f);
+    sts128(rowaddr + (((4 * h + c) ^ (row & 7u)) << 4), u);
   }
 }
 
 // Writes 32 floats into one 128-byte swizzled fp32 row (logical chunk c holds
 // elements 4c..4c+3).
-__device__ __forceinline__ void store_row_f32(uint8_t* rowp, uint32_t row, const float* x) {
+__device__ __forceinline__ void store_row_f32(uint32_t rowaddr, uint32_t row,
+                                              const uint32_t (&x)[32]) {
 #pragma unroll
   for (uint32_t c = 0; c < 8; ++c)
-    *reinterpret_cast<float4*>(rowp + ((c ^ (row & 7u)) << 4)) =
-        make_float4(x[4 * c + 0], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+    sts128(rowaddr + ((c ^ (row & 7u)) << 4),
+           make_uint4(x[4 * c + 0], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]));
 }
 
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* x) {
-  uint32_t a[32], b[32];
-  tmem_ld32(taddr, a);
-  tmem_ld32(taddr + 32, b);
-  tmem_wait_ld();
+__device__ __forceinline__ void tmem_st32_scaled(uint32_t taddr, const uint32_t (&x)[32], float f) {
+  uint32_t a[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    x[i] = __uint_as_float(a[i]);
-    x[32 + i] = __uint_as_float(b[i]);
-  }
-}
-
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const float* x, float f) {
-  uint32_t a[32], b[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    a[i] = __float_as_uint(x[i] * f);
-    b[i] = __float_as_uint(x[32 + i] * f);
-  }
+  for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(x[i]) * f);
   tmem_st32(taddr, a);
-  tmem_st32(taddr + 32, b);
 }
 
+// ---------------------------------------------------------------------------
+// Context, failure handling, bounded waits
+// ---------------------------------------------------------------------------
 struct Ctx {
   uint8_t* sm;
+  uint32_t sbase;           // shared-space address of sm
   uint64_t* bar;
-  float* gpow;
   volatile uint32_t* misc;  // [0] TMEM base, [1..2] work slots, [3] abort
   uint32_t tmem;
 };
 
 __device__ __forceinline__ bool aborted(const Ctx& c) { return c.misc[3] != 0; }
 
-__device__ __noinline__ void fail(const Ctx& c, const Params& p, int code) {
+__device__ __forceinline__ void fail(const Ctx& c, const Params& p, int code) {
   c.misc[3] = 1;
   atomicOr(p.status, code);
 }
 
-// Bounded wait; on time-out records the failure and returns false.
+// Bounded wait (single-thread roles); on time-out records the failure.
 __device__ __forceinline__ bool wait_bar(const Ctx& c, const Params& p, int id, uint32_t parity) {
   if (aborted(c)) return false;
   if (mbar_wait(&c.bar[id], parity, p.wait_limit_ns)) return true;
@@ -196,8 +242,8 @@ __device__ __forceinline__ bool wait_bar(const Ctx& c, const Params& p, int id, 
   return false;
 }
 
-// Warp-uniform bounded wait for the compute warps: all 32 lanes take the same
-// branch, so warp-collective tcgen05.ld/st that follow are never split.
+// Warp-uniform bounded wait for the compute groups: all 32 lanes take the same
+// branch, so the warp-collective tcgen05.ld/st that follow are never split.
 __device__ __forceinline__ bool cwait(const Ctx& c, const Params& p, int id, uint32_t parity) {
   bool ok = !aborted(c) && mbar_wait(&c.bar[id], parity, p.wait_limit_ns);
   ok = __all_sync(0xffffffffu, ok);
@@ -205,16 +251,16 @@ __device__ __forceinline__ bool cwait(const Ctx& c, const Params& p, int id, uin
   return ok;
 }
 
-// Synchronisation of the 256 compute threads through an mbarrier (bounded,
-// unlike bar.sync, so a failed wait elsewhere cannot hang the others).
-__device__ __forceinline__ bool csync(const Ctx& c, const Params& p, uint32_t& n) {
-  mbar_arrive(&c.bar[B_CSYNC]);
-  return cwait(c, p, B_CSYNC, n++ & 1u);
+// Synchronises the threads of one compute group through an mbarrier
+// (bounded, unlike bar.sync, so a failed wait elsewhere cannot hang the group).
+__device__ __forceinline__ bool gsync(const Ctx& c, const Params& p, int id, uint32_t& n) {
+  mbar_arrive(&c.bar[id]);
+  return cwait(c, p, id, n++ & 1u);
 }
 
 // Next work item: dynamic ticket for chunked runs, static stride otherwise.
 __device__ __forceinline__ int next_work(const Params& p, int& static_next) {
-  if (p.nchunks > 1) return atomicAdd(p.ticket, 1);
+  if (p.nchunks > 1) return p.ticket_base + atomicAdd(p.ticket, 1);
   const int w = static_next;
   static_next += gridDim.x;
   return w;
@@ -234,6 +280,7 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
     const uint32_t s = it & 1u;
     if (it >= 2 && !wait_bar(c, p, ring_e + s, ((it >> 1) - 1) & 1u)) return false;
     uint8_t* dst = c.sm + off + s * TILE;
+    LA_TRACE_EVENT(ring_f == B_QF ? 0 : ring_f == B_KF ? 1 : 2, it);
     mbar_arrive_expect_tx(&c.bar[ring_f + s], TILE);
     tma_load_3d(dst, tm, &c.bar[ring_f + s], 0, row, seq, pol);
     tma_load_3d(dst + PLANE, tm, &c.bar[ring_f + s], 64, row, seq, pol);
@@ -242,11 +289,14 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
   };
   // Before leaving, wait (bounded) for every load still in flight so no TMA
   // write lands in shared memory after the CTA exits.
+  auto drain_ring = [&](int ring_f, uint32_t n) {
+    for (uint32_t j = n >= 2 ? n - 2 : 0; j < n; ++j)
+      mbar_wait(&c.bar[ring_f + (j & 1u)], (j >> 1) & 1u, p.wait_limit_ns);
+  };
   auto drain = [&]() {
-    const uint32_t rings[3][2] = {{B_QF, q_it}, {B_KF, k_it}, {B_VF, v_it}};
-    for (int r = 0; r < 3; ++r)
-      for (uint32_t j = rings[r][1] >= 2 ? rings[r][1] - 2 : 0; j < rings[r][1]; ++j)
-        mbar_wait(&c.bar[rings[r][0] + (j & 1u)], (j >> 1) & 1u, p.wait_limit_ns);
+    drain_ring(B_QF, q_it);
+    drain_ring(B_KF, k_it);
+    drain_ring(B_VF, v_it);
   };
   for (;;) {
     const int w = next_work(p, static_next);
@@ -283,18 +333,19 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
   constexpr uint32_t ID_KMAJ = idesc_bf16_f32(128, 128, false, false);  // Q K^T
   constexpr uint32_t ID_BMN = idesc_bf16_f32(128, 128, false, true);    // Q~ S, P V
   constexpr uint32_t ID_AMN = idesc_bf16_f32(128, 128, true, true);     // K~^T V
-  const uint32_t sbase = smem_u32(c.sm);
+  const uint32_t sbase = c.sbase;
   const uint32_t kvb = sbase + OFF_KVB;
   uint32_t q_it = 0, k_it = 0, v_it = 0, w_it = 0, gb = 0;
   uint32_t ready_n = 0, kvb_n = 0, kvfree_n = 0;
   uint32_t kt_n[2] = {0, 0};
 
-  // S/P buffer (gb & 1) <- Q K^T for phase-2 block gidx of the current item.
+  // S/P buffer (gidx & 1) <- Q K^T for global phase-2 block gidx.
   auto issue_S = [&](uint32_t qi, uint32_t ki, uint32_t gidx) -> bool {
     const uint32_t qs = qi & 1u, ks = ki & 1u, buf = gidx & 1u;
     if (!wait_bar(c, p, B_QF + qs, (qi >> 1) & 1u)) return false;
     if (!wait_bar(c, p, B_KF + ks, (ki >> 1) & 1u)) return false;
     if (gidx >= 2 && !wait_bar(c, p, B_SE + buf, ((gidx >> 1) - 1) & 1u)) return false;
+    LA_TRACE_EVENT(4, gidx);
     tc_fence_after();
     const uint32_t qa = sbase + OFF_Q + qs * TILE, ka = sbase + OFF_K + ks * TILE;
 #pragma unroll
@@ -333,18 +384,24 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
         ++v_it;
       }
       mma_commit(&c.bar[B_AGG_FULL]);
+      LA_TRACE_EVENT(21, w_it);
     }
     const uint32_t q0 = q_it, k0 = k_it, v0 = v_it, g0 = gb;
     const uint32_t nb = static_cast<uint32_t>(it.nb);
     if (!issue_S(q0, k0, g0)) return;
     for (uint32_t n = 0; n < nb; ++n) {
       const uint32_t g = g0 + n;
-      const uint32_t qs = (q0 + n) & 1u, ks = (k0 + n) & 1u, vs = (v0 + n) & 1u;
+      const uint32_t ks = (k0 + n) & 1u, vs = (v0 + n) & 1u;
       if (!wait_bar(c, p, B_READY, ready_n++ & 1u)) return;
+      LA_TRACE_EVENT(3, g);
+      // the next block's scores first, so group X can start on them
+      if (n + 1 < nb && !issue_S(q0 + n + 1, k0 + n + 1, g + 1)) return;
       if (!wait_bar(c, p, B_KVB_READY, kvb_n++ & 1u)) return;
+      LA_TRACE_EVENT(5, g);
       if (!wait_bar(c, p, B_VF + vs, ((v0 + n) >> 1) & 1u)) return;
+      LA_TRACE_EVENT(6, g);
       tc_fence_after();
-      const uint32_t qa = sbase + OFF_Q + qs * TILE, ka = sbase + OFF_K + ks * TILE;
+      const uint32_t ka = sbase + OFF_K + ks * TILE;
       const uint32_t va = sbase + OFF_V + vs * TILE;
       // state += (decayed K)^T V
 #pragma unroll
@@ -352,27 +409,26 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
         mma_ss(c.tmem + TM_KV, sdesc_sw128(ka + kk * 2048u, PLANE, 1024),
                sdesc_sw128(va + kk * 2048u, PLANE, 1024), ID_AMN, 1);
       if (g >= 1 && !wait_bar(c, p, B_O_EMPTY, (g - 1) & 1u)) return;
+      LA_TRACE_EVENT(7, g);
       tc_fence_after();
-      // O = (gamma^(i+1) Q) S_bf16
-#pragma unroll
-      for (uint32_t kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * PLANE + (kk & 3u) * 32u;
-        mma_ss(c.tmem + TM_O, sdesc_sw128(qa + off, 16, 1024),
-               sdesc_sw128(kvb + kk * 2048u, PLANE, 1024), ID_BMN, kk > 0);
-      }
-      // Q and K tiles are dead once the state update and the inter term finish.
-      mma_commit(&c.bar[B_KVO_DONE]);
-      mma_commit(&c.bar[B_QE + qs]);
-      mma_commit(&c.bar[B_KE + ks]);
-      // O += P V, P read from TMEM (bf16 pairs in the S buffer)
+      // O = (gamma^(i+1) Q) S_bf16, the decayed Q read from TMEM
+      const uint32_t abase = c.tmem + TM_S0 + (g & 1u) * 128u;
 #pragma unroll
       for (uint32_t kk = 0; kk < 8; ++kk)
-        mma_ts(c.tmem + TM_O, c.tmem + TM_S0 + (g & 1u) * 128u + kk * 8u,
+        mma_ts(c.tmem + TM_O, abase + 32u + (kk >> 2) * 64u + (kk & 3u) * 8u,
+               sdesc_sw128(kvb + kk * 2048u, PLANE, 1024), ID_BMN, kk > 0);
+      // The K tile is dead once the state update finishes.
+      mma_commit(&c.bar[B_KVO_DONE]);
+      mma_commit(&c.bar[B_KE + ks]);
+      // O += P V, P read from TMEM (bf16 pairs: j < 64 at +0, j >= 64 at +64)
+#pragma unroll
+      for (uint32_t kk = 0; kk < 8; ++kk)
+        mma_ts(c.tmem + TM_O, abase + (kk >> 2) * 64u + (kk & 3u) * 8u,
                sdesc_sw128(va + kk * 2048u, PLANE, 1024), ID_BMN, 1);
       mma_commit(&c.bar[B_O_FULL]);
       mma_commit(&c.bar[B_SE + (g & 1u)]);
-      // The V tile is released by the epilogue after it has staged the output there.
-      if (n + 1 < nb && !issue_S(q0 + n + 1, k0 + n + 1, g + 1)) return;
+      LA_TRACE_EVENT(8, g);
+      // The V tile is released by group Y after it has staged the output there.
     }
     q_it += nb;
     k_it += nb;
@@ -390,81 +446,17 @@ __device__ void mma_issuer(const Ctx& c, const Params& p) {
 }
 
 // ---------------------------------------------------------------------------
-// Compute warps (256 threads): thread owns TMEM lane / tile row r and the
-// column half hf (64 columns) of that row.
+// Group X: decay-causal mask and the in-place operand decays.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void load_row64(const float* src, float* x) {
-  const float4* s4 = reinterpret_cast<const float4*>(src);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float4 v = __ldcg(s4 + i);
-    x[4 * i] = v.x;
-    x[4 * i + 1] = v.y;
-    x[4 * i + 2] = v.z;
-    x[4 * i + 3] = v.w;
-  }
-}
-
-__device__ __forceinline__ void store_row64(float* dst, const float* x) {
-  float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-    __stcg(d4 + i, make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]));
-}
-
-// Entering state of a work item: zero, the caller's initial state, or the
-// inclusive state published by the previous chunk.  Returns false on failure.
-__device__ bool entering_state(const Ctx& c, const Params& p, const Item& it, uint32_t tid,
-                               int64_t row_off, uint32_t& csync_n, float* prev) {
-  if (it.chunk > 0) {
-    const int slot = (it.chunk - 1) & 1;
-    if (tid == 0) {
-      const int* flag = p.flags + it.seq * 2 + slot;
-      const uint64_t t0 = globaltimer_ns();
-      uint32_t spins = 0;
-      while (ld_acquire_gpu(flag) != it.chunk) {
-        if ((++spins & 15u) == 0 &&
-            (aborted(c) || globaltimer_ns() - t0 > p.wait_limit_ns)) {
-          fail(c, p, 2);
-          break;
-        }
-      }
-    }
-    if (!csync(c, p, csync_n)) return false;
-    load_row64(p.prefix + (static_cast<int64_t>(it.seq) * 2 + slot) * (HD * HD) + row_off, prev);
-  } else if (p.init_state) {
-    load_row64(p.init_state + static_cast<int64_t>(it.seq) * (HD * HD) + row_off, prev);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 64; ++i) prev[i] = 0.f;
-  }
-  return true;
-}
-
-__device__ void compute(const Ctx& c, const Params& p, const CUtensorMap* to) {
-  const uint32_t tid = threadIdx.x;  // 0..255
-  const uint32_t warp = tid >> 5;
-  const uint32_t r = (warp & 3u) * 32u + (tid & 31u);
-  const int ri = static_cast<int>(r);
+__device__ void group_x(const Ctx& c, const Params& p) {
+  const uint32_t t = threadIdx.x - 32u * X_WARP0;  // 0..255
+  const uint32_t warp = t >> 5;
+  const uint32_t r = (warp & 3u) * 32u + (t & 31u);
   const uint32_t hf = warp >> 2;
   const uint32_t lane_base = ((warp & 3u) * 32u) << 16;
-  const uint32_t t_kv = c.tmem + lane_base + TM_KV + hf * 64u;
-  const uint32_t t_o = c.tmem + lane_base + TM_O + hf * 64u;
-  const int64_t row_off = static_cast<int64_t>(r) * HD + hf * 64;
-  const uint64_t pol_out = policy_evict_first();
-  uint32_t q_it = 0, k_it = 0, v_it = 0, w_it = 0, gb = 0, agg_n = 0, csync_n = 0;
-  // V slot whose staged output the last TMA stores may still read (thread 0)
-  int pend_v = -1;
-  auto release_pending = [&]() {
-    if (tid == 0 && pend_v >= 0) {
-      bulk_wait_group_read<0>();
-      mbar_arrive(&c.bar[B_VE + pend_v]);
-      pend_v = -1;
-    }
-  };
-
-  bool ok = true;
-  while (ok) {
+  const uint32_t gtab = c.sbase + OFF_GTAB;
+  uint32_t q_it = 0, k_it = 0, w_it = 0, gb = 0, xs_n = 0;
+  for (;;) {
     const uint32_t ws = w_it & 1u;
     if (!cwait(c, p, B_WF + ws, (w_it >> 1) & 1u)) break;
     const int w = static_cast<int>(c.misc[1 + ws]);
@@ -474,150 +466,317 @@ __device__ void compute(const Ctx& c, const Params& p, const CUtensorMap* to) {
     const Item it = decode_item(p, w);
     const float lam = p.slopes[it.seq % p.H];
 
-    if (!csync(c, p, csync_n)) break;  // the previous item's table is no longer read
-    if (tid <= BLK) c.gpow[tid] = expf(-lam * static_cast<float>(tid));
-    if (!csync(c, p, csync_n)) break;
-    mbar_arrive(&c.bar[B_KV_FREE]);
+    // decay table: gtab[u] = gamma^(127-u) for u <= 127, 0 above (the causal mask)
+    if (!gsync(c, p, B_XSYNC, xs_n)) break;  // the previous item's table is no longer read
+    sts32f(gtab + 4u * t, t <= 127u ? expf(-lam * static_cast<float>(127u - t)) : 0.f);
+    if (!gsync(c, p, B_XSYNC, xs_n)) break;
 
-    // ---- phase 1: local chunk state from decayed K ----
-    if (it.phase1) {
+    bool ok = true;
+    if (it.phase1) {  // K rows decayed to the chunk end: gamma^(Lc-1-j)
       for (int b = 0; b < it.nb && ok; ++b) {
         const uint32_t ks = k_it & 1u;
         if (!cwait(c, p, B_KF + ks, (k_it >> 1) & 1u)) { ok = false; break; }
-        const int jc = b * BLK + ri;
+        const int jc = b * BLK + static_cast<int>(r);
         const float f = jc < it.Lc ? expf(-lam * static_cast<float>(it.Lc - 1 - jc)) : 0.f;
-        scale_row(c.sm + OFF_K + ks * TILE + hf * PLANE + r * 128u, r, f);
+        scale_row(c.sbase + OFF_K + ks * TILE + hf * PLANE + r * 128u, r, f);
         fence_proxy_async_smem();
         mbar_arrive(&c.bar[B_KT + ks]);
+        if (t == 0) LA_TRACE_EVENT(22, k_it);
         ++k_it;
-        ++v_it;
       }
-      if (!ok) break;
     }
-
-    // ---- entering state; publication of this chunk's inclusive state ----
-    {
-      float prev[64];
-      if (!entering_state(c, p, it, tid, row_off, csync_n, prev)) break;
-      if (it.phase1) {
-        if (!cwait(c, p, B_AGG_FULL, agg_n++ & 1u)) break;
-        tc_fence_after();
-        float agg[64];
-        tmem_ld64(t_kv, agg);
-        const float gL = expf(-lam * static_cast<float>(it.Lc));
-#pragma unroll
-        for (int i = 0; i < 64; ++i) agg[i] = fmaf(gL, prev[i], agg[i]);
-        store_row64(p.prefix + (static_cast<int64_t>(it.seq) * 2 + (it.chunk & 1)) * (HD * HD) +
-                        row_off,
-                    agg);
-        __threadfence();
-        if (!csync(c, p, csync_n)) break;
-        if (tid == 0) st_release_gpu(p.flags + it.seq * 2 + (it.chunk & 1), it.chunk + 1);
-      }
-      // state for block 0: bf16 copy for the MMA, fp32 copy decayed by gamma^len0
-      store_row_bf16(c.sm + OFF_KVB + hf * PLANE + r * 128u, r, prev);
-      tmem_st64(t_kv, prev, c.gpow[min(BLK, it.Lc)]);
-      fence_proxy_async_smem();
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&c.bar[B_KVB_READY]);
-    }
-
-    // ---- phase 2: blocked form from the entering state ----
-    for (int n = 0; n < it.nb; ++n) {
+    for (int n = 0; n < it.nb && ok; ++n) {
       const uint32_t g = gb;
       const int len = min(BLK, it.Lc - n * BLK);
-      const uint32_t qs = q_it & 1u, ks = k_it & 1u, vs = v_it & 1u;
-      uint8_t* qtile = c.sm + OFF_Q + qs * TILE;
-      uint8_t* ktile = c.sm + OFF_K + ks * TILE;
-      uint8_t* vtile = c.sm + OFF_V + vs * TILE;
-      const uint32_t t_s = c.tmem + lane_base + TM_S0 + (g & 1u) * 128u;
-
-      // (A) decay-causal mask of Q K^T into P (bf16, TMEM); gamma^(i+1) Q and
-      //     gamma^(len-1-j) K in place in shared memory.
+      const uint32_t qs = q_it & 1u, ks = k_it & 1u;
       if (!cwait(c, p, B_SF + (g & 1u), (g >> 1) & 1u) ||
           !cwait(c, p, B_QF + qs, (q_it >> 1) & 1u) ||
           !cwait(c, p, B_KF + ks, (k_it >> 1) & 1u)) { ok = false; break; }
+      if (t == 0) LA_TRACE_EVENT(9, g);
       tc_fence_after();
-      {
-        float sv[64];
-        tmem_ld64(t_s + hf * 64u, sv);
-        uint32_t pk[32];
+      const uint32_t t_s = c.tmem + lane_base + TM_S0 + (g & 1u) * 128u + hf * 64u;
+      // P_ij = S_ij * gtab[j - r + 127] (zero above the diagonal); rows past len
+      // have zero scores (zero-filled Q), so they give zero P as well.  In the
+      // quarter with every column above every row (hf = 1, rows < 64) P is 0.
+      uint32_t pk[32];
+      if (hf == 1 && (warp & 3u) < 2) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int j0 = static_cast<int>(hf) * 64 + 2 * i;
-          const float p0 = (j0 <= ri && ri < len) ? sv[2 * i] * c.gpow[ri - j0] : 0.f;
-          const float p1 = (j0 + 1 <= ri && ri < len) ? sv[2 * i + 1] * c.gpow[ri - j0 - 1] : 0.f;
-          pk[i] = pack_bf16x2(p0, p1);
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
+      } else {
+#pragma unroll
+        for (uint32_t half = 0; half < 2; ++half) {
+          uint32_t sc[32];
+          tmem_ld32(t_s + half * 32u, sc);
+          const uint32_t u0 = gtab + 4u * (hf * 64u + half * 32u + 127u - r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[16 * half + i] = pack_bf16x2(__uint_as_float(sc[2 * i]) * lds32f(u0 + 8u * i),
+                                            __uint_as_float(sc[2 * i + 1]) * lds32f(u0 + 8u * i + 4u));
         }
-        // every S column is in registers before P (half as many columns) overwrites it
-        if (!csync(c, p, csync_n)) { ok = false; break; }
-        tmem_st32(t_s + hf * 32u, pk);
       }
-      scale_row(qtile + hf * PLANE + r * 128u, r, ri < len ? c.gpow[ri + 1] : 0.f);
-      scale_row(ktile + hf * PLANE + r * 128u, r, ri < len ? c.gpow[len - 1 - ri] : 0.f);
+      tmem_st32(t_s, pk);
+      // gamma^(r+1) Q (bf16) into the S buffer's free columns; the Q tile is then dead
+      {
+        const float fq = lds32f(gtab + 4u * (127u - r)) * lds32f(gtab + 4u * 126u);
+        const uint32_t qrow = c.sbase + OFF_Q + qs * TILE + hf * PLANE + r * 128u;
+        uint32_t qv[32];
+#pragma unroll
+        for (uint32_t ch = 0; ch < 8; ++ch) {
+          const uint4 x = lds128(qrow + ((ch ^ (r & 7u)) << 4));
+          qv[4 * ch + 0] = scale_bf16x2(x.x, fq);
+          qv[4 * ch + 1] = scale_bf16x2(x.y, fq);
+          qv[4 * ch + 2] = scale_bf16x2(x.z, fq);
+          qv[4 * ch + 3] = scale_bf16x2(x.w, fq);
+        }
+        mbar_arrive(&c.bar[B_QE + qs]);
+        tmem_st32(t_s + 32u, qv);
+      }
+      // gamma^(len-1-r) K (0 past len) in place
+      const float fk = lds32f(gtab + 4u * (128u - static_cast<uint32_t>(len) + r));
+      scale_row(c.sbase + OFF_K + ks * TILE + hf * PLANE + r * 128u, r, fk);
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&c.bar[B_READY]);
-      release_pending();
+      if (t == 0) LA_TRACE_EVENT(10, g);
+      ++q_it;
+      ++k_it;
+      ++gb;
+    }
+    if (!ok) break;
+  }
+}
 
-      // (B) state: bf16 copy for the next block's inter term, then decay in TMEM
+// ---------------------------------------------------------------------------
+// Group Y: state copy/decay, chunk scan, epilogue.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ld_global32(const float* src, uint32_t (&x)[32]) {
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 v = __ldcg(s4 + i);
+    x[4 * i] = __float_as_uint(v.x);
+    x[4 * i + 1] = __float_as_uint(v.y);
+    x[4 * i + 2] = __float_as_uint(v.z);
+    x[4 * i + 3] = __float_as_uint(v.w);
+  }
+}
+
+__device__ __forceinline__ void st_global32(float* dst, const uint32_t (&x)[32]) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    __stcg(d4 + i, make_float4(__uint_as_float(x[4 * i]), __uint_as_float(x[4 * i + 1]),
+                               __uint_as_float(x[4 * i + 2]), __uint_as_float(x[4 * i + 3])));
+}
+
+// Chunk states in the scan scratch use a thread-blocked layout: the float4 that
+// thread (row r, half hf) holds as its i-th vector of pass h lives at float4
+// index ((hf * 2 + h) * 8 + i) * 128 + r, so each warp-wide access covers 512
+// contiguous bytes.
+__device__ __forceinline__ void ld_scan32(const float* base, uint32_t r, uint32_t hf, uint32_t h,
+                                          uint32_t (&x)[32]) {
+  const float4* s4 = reinterpret_cast<const float4*>(base);
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i) {
+    const float4 v = __ldcg(s4 + ((hf * 2u + h) * 8u + i) * 128u + r);
+    x[4 * i] = __float_as_uint(v.x);
+    x[4 * i + 1] = __float_as_uint(v.y);
+    x[4 * i + 2] = __float_as_uint(v.z);
+    x[4 * i + 3] = __float_as_uint(v.w);
+  }
+}
+
+__device__ __forceinline__ void st_scan32(float* base, uint32_t r, uint32_t hf, uint32_t h,
+                                          const uint32_t (&x)[32]) {
+  float4* d4 = reinterpret_cast<float4*>(base);
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i)
+    __stcg(d4 + ((hf * 2u + h) * 8u + i) * 128u + r,
+           make_float4(__uint_as_float(x[4 * i]), __uint_as_float(x[4 * i + 1]),
+                       __uint_as_float(x[4 * i + 2]), __uint_as_float(x[4 * i + 3])));
+}
+
+__device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
+  const uint32_t t = threadIdx.x - 32u * Y_WARP0;  // 0..127
+  const uint32_t r = t;                            // TMEM lane / tile row
+  const uint32_t lane_base = ((t >> 5) * 32u) << 16;
+  const uint32_t t_kv = c.tmem + lane_base + TM_KV;
+  const uint32_t t_o = c.tmem + lane_base + TM_O;
+  const int64_t row_off = static_cast<int64_t>(r) * HD;
+  const bool leader = (t == 0);
+  const uint64_t pol_out = policy_evict_first();
+  uint32_t v_it = 0, w_it = 0, gb = 0, agg_n = 0, ys_n = 0;
+  // kvb row address of column quarter q (32 columns): plane q / 2, chunks 4 (q % 2)..
+  auto kvb_row = [&](uint32_t q) { return c.sbase + OFF_KVB + (q >> 1) * PLANE + r * 128u; };
+
+  for (;;) {
+    const uint32_t ws = w_it & 1u;
+    if (!cwait(c, p, B_WF + ws, (w_it >> 1) & 1u)) break;
+    const int w = static_cast<int>(c.misc[1 + ws]);
+    mbar_arrive(&c.bar[B_WE + ws]);
+    ++w_it;
+    if (w >= p.total) break;
+    const Item it = decode_item(p, w);
+    const float lam = p.slopes[it.seq % p.H];
+    mbar_arrive(&c.bar[B_KV_FREE]);  // done with the previous item's state
+    if (leader) LA_TRACE_EVENT(15, w_it);
+    if (it.phase1) v_it += it.nb;
+
+    // ---- entering state; publication of this chunk's inclusive state ----
+    const float* scan_src = nullptr;  // previous chunk's state (scan layout)
+    const float* init_src = nullptr;  // caller's initial state (row layout)
+    if (it.chunk > 0) {
+      const int slot = (it.chunk - 1) & 1;
+      if (leader) {
+        const int* flag = p.flags + it.seq * 2 + slot;
+        const uint64_t t0 = globaltimer_ns();
+        uint32_t spins = 0;
+        while (ld_acquire_gpu(flag) != it.chunk) {
+          if ((++spins & 15u) == 0 && (aborted(c) || globaltimer_ns() - t0 > p.wait_limit_ns)) {
+            fail(c, p, 2);
+            break;
+          }
+        }
+      }
+      if (!gsync(c, p, B_YSYNC, ys_n)) break;
+      scan_src = p.prefix + (static_cast<int64_t>(it.seq) * 2 + slot) * (HD * HD);
+    } else if (p.init_state) {
+      init_src = p.init_state + static_cast<int64_t>(it.seq) * (HD * HD) + row_off;
+    }
+    if (leader) LA_TRACE_EVENT(16, w_it);
+    if (it.phase1 && !cwait(c, p, B_AGG_FULL, agg_n++ & 1u)) break;
+    if (leader) LA_TRACE_EVENT(17, w_it);
+    tc_fence_after();
+    {
+      const float gL = expf(-lam * static_cast<float>(it.Lc));
+      const float g0 = expf(-lam * static_cast<float>(min(BLK, it.Lc)));
+      float* pub = p.prefix + (static_cast<int64_t>(it.seq) * 2 + (it.chunk & 1)) * (HD * HD);
+#pragma unroll 1
+      for (uint32_t q = 0; q < 4; ++q) {
+        uint32_t prev[32];
+        if (scan_src) {
+          ld_scan32(scan_src, r, q >> 1, q & 1u, prev);
+        } else if (init_src) {
+          ld_global32(init_src + 32 * q, prev);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) prev[i] = 0u;
+        }
+        if (it.phase1) {
+          uint32_t agg[32];
+          tmem_ld32(t_kv + 32u * q, agg);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            agg[i] = __float_as_uint(fmaf(gL, __uint_as_float(prev[i]), __uint_as_float(agg[i])));
+          st_scan32(pub, r, q >> 1, q & 1u, agg);
+        }
+        store_half_bf16(kvb_row(q), r, q & 1u, prev, 1.f);
+        tmem_st32_scaled(t_kv + 32u * q, prev, g0);
+      }
+    }
+    if (leader) LA_TRACE_EVENT(18, w_it);
+    if (it.phase1) {
+      // the group's stores are ordered before the leader's fence and release
+      if (!gsync(c, p, B_YSYNC, ys_n)) break;
+      if (leader) {
+        __threadfence();
+        st_release_gpu(p.flags + it.seq * 2 + (it.chunk & 1), it.chunk + 1);
+      }
+    }
+    if (leader) LA_TRACE_EVENT(19, w_it);
+    fence_proxy_async_smem();
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(&c.bar[B_KVB_READY]);
+    if (leader) LA_TRACE_EVENT(20, w_it);
+
+    bool ok = true;
+    for (int n = 0; n < it.nb && ok; ++n) {
+      const uint32_t g = gb;
+      const uint32_t vs = v_it & 1u;
+      // (B) state: bf16 copy for the next block's inter term, decay in TMEM
       if (!cwait(c, p, B_KVO_DONE, g & 1u)) { ok = false; break; }
+      if (leader) LA_TRACE_EVENT(11, g);
       tc_fence_after();
       {
-        float kv[64];
-        tmem_ld64(t_kv, kv);
-        if (n + 1 < it.nb) {
-          store_row_bf16(c.sm + OFF_KVB + hf * PLANE + r * 128u, r, kv);
-          tmem_st64(t_kv, kv, c.gpow[min(BLK, it.Lc - (n + 1) * BLK)]);
+        const bool more = n + 1 < it.nb;
+        const float gnext =
+            more ? expf(-lam * static_cast<float>(min(BLK, it.Lc - (n + 1) * BLK))) : 1.f;
+        const bool fin = !more && p.final_state && it.chunk + 1 == p.nchunks;
+#pragma unroll 1
+        for (uint32_t q = 0; q < 4; ++q) {
+          uint32_t kv[32];
+          tmem_ld32(t_kv + 32u * q, kv);
+          tmem_wait_ld();
+          if (more) {
+            store_half_bf16(kvb_row(q), r, q & 1u, kv, 1.f);
+            tmem_st32_scaled(t_kv + 32u * q, kv, gnext);
+          } else if (fin) {
+            st_global32(p.final_state + static_cast<int64_t>(it.seq) * (HD * HD) + row_off + 32 * q,
+                        kv);
+          }
+        }
+        if (more) {
           fence_proxy_async_smem();
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&c.bar[B_KVB_READY]);
-        } else if (p.final_state && it.chunk + 1 == p.nchunks) {
-          store_row64(p.final_state + static_cast<int64_t>(it.seq) * (HD * HD) + row_off, kv);
         }
+        if (leader) LA_TRACE_EVENT(12, g);
       }
-
       // (C) epilogue: O -> swizzled staging in this block's V slot (dead once O
       //     is complete), 64 columns at a time -> TMA store.
       if (!cwait(c, p, B_O_FULL, g & 1u)) { ok = false; break; }
+      if (leader) LA_TRACE_EVENT(13, g);
       tc_fence_after();
-      {
-        float o[64];
-        tmem_ld64(t_o, o);
-        tc_fence_before();
-        mbar_arrive(&c.bar[B_O_EMPTY]);
-        const int row = it.t0 + n * BLK;
-        for (uint32_t half = 0; half < 2 && ok; ++half) {
-          if (hf == half) {
-            store_row_f32(vtile + r * 128u, r, o);
-            store_row_f32(vtile + PLANE + r * 128u, r, o + 32);
-          }
-          fence_proxy_async_smem();
-          if (!csync(c, p, csync_n)) { ok = false; break; }
-          if (tid == 0) {
-            tma_store_3d(to, vtile, 64 * half, row, it.seq, pol_out);
-            tma_store_3d(to, vtile + PLANE, 64 * half + 32, row, it.seq, pol_out);
-            bulk_commit_group();
-            if (half == 0) bulk_wait_group_read<0>();
-          }
-          if (half == 0 && !csync(c, p, csync_n)) { ok = false; break; }
-        }
-        if (tid == 0) pend_v = static_cast<int>(vs);
+      const uint32_t vtile = c.sbase + OFF_V + vs * TILE;
+      const uint8_t* vtile_g = c.sm + OFF_V + vs * TILE;
+      const int row = it.t0 + n * BLK;
+      uint32_t o0[32], o1[32];
+      tmem_ld32(t_o, o0);
+      tmem_ld32(t_o + 32u, o1);
+      tmem_wait_ld();
+      store_row_f32(vtile + r * 128u, r, o0);
+      store_row_f32(vtile + PLANE + r * 128u, r, o1);
+      fence_proxy_async_smem();
+      if (!gsync(c, p, B_YSYNC, ys_n)) { ok = false; break; }
+      if (leader) {
+        tma_store_3d(to, vtile_g, 0, row, it.seq, pol_out);
+        tma_store_3d(to, vtile_g + PLANE, 32, row, it.seq, pol_out);
+        bulk_commit_group();
       }
-      if (!ok) break;
-      ++q_it;
-      ++k_it;
+      tmem_ld32(t_o + 64u, o0);
+      tmem_ld32(t_o + 96u, o1);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&c.bar[B_O_EMPTY]);
+      if (leader) bulk_wait_group_read<0>();
+      if (!gsync(c, p, B_YSYNC, ys_n)) { ok = false; break; }
+      store_row_f32(vtile + r * 128u, r, o0);
+      store_row_f32(vtile + PLANE + r * 128u, r, o1);
+      fence_proxy_async_smem();
+      if (!gsync(c, p, B_YSYNC, ys_n)) { ok = false; break; }
+      if (leader) {
+        tma_store_3d(to, vtile_g, 64, row, it.seq, pol_out);
+        tma_store_3d(to, vtile_g + PLANE, 96, row, it.seq, pol_out);
+        bulk_commit_group();
+        bulk_wait_group_read<0>();
+        mbar_arrive(&c.bar[B_VE + vs]);
+      }
+      if (leader) LA_TRACE_EVENT(14, g);
       ++v_it;
       ++gb;
     }
-    release_pending();
+    if (!ok) break;
   }
-  if (tid == 0) bulk_wait_group<0>();
+  if (leader) bulk_wait_group<0>();
 }
 
+// 14 warps on 4 SM sub-partitions (16K registers each, at most 4 warps on one)
+// leave up to 128 registers per thread.
 __global__ void __launch_bounds__(THREADS, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
@@ -626,15 +785,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   Ctx c;
   c.sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                     ~static_cast<uintptr_t>(1023));
+  c.sbase = smem_u32(c.sm);
   c.bar = reinterpret_cast<uint64_t*>(c.sm + OFF_BAR);
-  c.gpow = reinterpret_cast<float*>(c.sm + OFF_GPOW);
   c.misc = reinterpret_cast<volatile uint32_t*>(c.sm + OFF_MISC);
   const uint32_t warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&c.bar[B_QF + i], 1);
-      mbar_init(&c.bar[B_QE + i], 1);
+      mbar_init(&c.bar[B_QE + i], X_THREADS);
       mbar_init(&c.bar[B_KF + i], 1);
       mbar_init(&c.bar[B_KE + i], 1);
       mbar_init(&c.bar[B_VF + i], 1);
@@ -642,17 +801,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&c.bar[B_SF + i], 1);
       mbar_init(&c.bar[B_SE + i], 1);
       mbar_init(&c.bar[B_WF + i], 1);
-      mbar_init(&c.bar[B_WE + i], 1 + C_THREADS);
-      mbar_init(&c.bar[B_KT + i], C_THREADS);
+      mbar_init(&c.bar[B_WE + i], 1 + X_THREADS + Y_THREADS);
+      mbar_init(&c.bar[B_KT + i], X_THREADS);
     }
-    mbar_init(&c.bar[B_READY], C_THREADS);
-    mbar_init(&c.bar[B_KVB_READY], C_THREADS);
+    mbar_init(&c.bar[B_READY], X_THREADS);
+    mbar_init(&c.bar[B_KVB_READY], Y_THREADS);
     mbar_init(&c.bar[B_KVO_DONE], 1);
     mbar_init(&c.bar[B_O_FULL], 1);
-    mbar_init(&c.bar[B_O_EMPTY], C_THREADS);
+    mbar_init(&c.bar[B_O_EMPTY], Y_THREADS);
     mbar_init(&c.bar[B_AGG_FULL], 1);
-    mbar_init(&c.bar[B_KV_FREE], C_THREADS);
-    mbar_init(&c.bar[B_CSYNC], C_THREADS);
+    mbar_init(&c.bar[B_KV_FREE], Y_THREADS);
+    mbar_init(&c.bar[B_XSYNC], X_THREADS);
+    mbar_init(&c.bar[B_YSYNC], Y_THREADS);
     mbar_init(&c.bar[B_DRAIN], 1);
     c.misc[3] = 0;
     fence_mbar_init();
@@ -677,8 +837,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == MMA_WARP) {
     if (lane_id() == 0) mma_issuer(c, p);
     __syncwarp();
+  } else if (warp < Y_WARP0) {
+    group_x(c, p);
   } else {
-    compute(c, p, &to);
+    group_y(c, p, &to);
   }
 
   tc_fence_before();

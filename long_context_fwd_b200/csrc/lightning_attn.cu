@@ -32,8 +32,17 @@ inline bool dims_ok(int B, int H, int N, int D, int E) {
   return n < (static_cast<__int128>(1) << 62) && static_cast<long long>(B) * H < (1ll << 31);
 }
 
+// Text of the CUDA error behind the calling thread's last LA_ERR_CUDA.
+thread_local const char* t_last_cuda_error = "no error";
+
+inline int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = cudaGetErrorString(e);
+  return LA_ERR_CUDA;
+}
+
 inline int launch_status() {
-  return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? LA_OK : cuda_fail(e);
 }
 
 inline int* status_word() {
@@ -50,16 +59,17 @@ int sm_count() {
   return n;
 }
 
-// Chunk length for the sequence split: whole sequences when there are enough
-// of them, else chunks of at most 1024 tokens (their K/V stay in L2 between the
-// two phases) so that the work items cover several waves of SMs.
+// Chunk length for the sequence split.  Whole sequences when there are at
+// least as many (b, h) problems as SMs (splitting costs a local-state pass and a
+// scan step per chunk); otherwise chunks of 1024-4096 tokens so that the work
+// items cover a few waves of SMs.
 int auto_chunk(int nseq, int N, int sms) {
   const int nblk = (N + 127) / 128;
-  if (nseq >= 4 * sms || nblk <= 4) return nblk * 128;
+  if (nseq >= sms || nblk <= 8) return nblk * 128;
   const int want_chunks = (4 * sms + nseq - 1) / nseq;
   int L = ((N + want_chunks - 1) / want_chunks + 127) / 128 * 128;
-  if (L < 512) L = 512;
-  if (L > 1024) L = 1024;
+  if (L < 1024) L = 1024;
+  if (L > 4096) L = 4096;
   return L;
 }
 
@@ -108,10 +118,12 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   if (nchunks > 1) {
     const size_t ctrl = ((static_cast<size_t>(nseq) * 2 + 1) * sizeof(int) + 255) / 256 * 256;
     const size_t bytes = ctrl + static_cast<size_t>(nseq) * 2 * 128 * 128 * sizeof(float);
-    if (cudaMallocAsync(&scratch, bytes, stream) != cudaSuccess) return LA_ERR_CUDA;
-    if (cudaMemsetAsync(scratch, 0, ctrl, stream) != cudaSuccess) {
+    cudaError_t e = cudaMallocAsync(&scratch, bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaMemsetAsync(scratch, 0, ctrl, stream);
+    if (e != cudaSuccess) {
       cudaFreeAsync(scratch, stream);
-      return LA_ERR_CUDA;
+      return cuda_fail(e);
     }
     p.ticket = static_cast<int*>(scratch);
     p.flags = p.ticket + 1;
@@ -119,19 +131,22 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   }
 
   // set on every call: the attribute belongs to the current device's context
-  const bool attr_ok =
+  const cudaError_t attr =
       cudaFuncSetAttribute(la::fwd::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           la::fwd::SMEM_BYTES) == cudaSuccess;
+                           la::fwd::SMEM_BYTES);
   int rc = LA_OK;
-  if (!attr_ok) {
-    rc = LA_ERR_CUDA;
+  if (attr != cudaSuccess) {
+    rc = cuda_fail(attr);
   } else {
     const int grid = static_cast<int>(total < sms ? total : sms);
     la::fwd::fwd_bf16_kernel<<<grid, la::fwd::THREADS, la::fwd::SMEM_BYTES, stream>>>(tq, tk, tv,
                                                                                     to, p);
     rc = launch_status();
   }
-  if (scratch && cudaFreeAsync(scratch, stream) != cudaSuccess) rc = LA_ERR_CUDA;
+  if (scratch) {
+    const cudaError_t e = cudaFreeAsync(scratch, stream);
+    if (e != cudaSuccess && rc == LA_OK) rc = cuda_fail(e);
+  }
   return rc;
 }
 
@@ -139,10 +154,10 @@ template <int D, int E>
 int launch_f32(const float* q, const float* k, const float* v, const float* slopes, float* out,
                int B, int H, int N, cudaStream_t stream) {
   constexpr size_t smem = la::fwd_f32_smem_bytes<D, E>();
-  const bool attr_ok =
+  const cudaError_t attr =
       cudaFuncSetAttribute(la::fwd_f32_kernel<D, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) == cudaSuccess;
-  if (!attr_ok) return LA_ERR_CUDA;
+                           static_cast<int>(smem));
+  if (attr != cudaSuccess) return cuda_fail(attr);
   la::fwd_f32_kernel<D, E><<<B * H, 256, smem, stream>>>(q, k, v, slopes, out, H, N);
   return launch_status();
 }
@@ -202,6 +217,17 @@ int lightning_attn_decode(const void* q, const void* k, const void* v, float* st
   return LA_ERR_UNSUPPORTED;
 }
 
+const char* lightning_attn_last_cuda_error(void) { return t_last_cuda_error; }
+
+#ifdef LA_TRACE
+// Tracing builds only: device buffer of TRACE_CTAS x TRACE_EVENTS x TRACE_SLOTS
+// u64 timestamps (or NULL to stop tracing).
+int lightning_attn_set_trace(unsigned long long* buf) {
+  const cudaError_t e = cudaMemcpyToSymbol(la::fwd::g_trace, &buf, sizeof(buf));
+  return e == cudaSuccess ? LA_OK : cuda_fail(e);
+}
+#endif
+
 const char* lightning_attn_status_string(int status) {
   switch (status) {
     case LA_OK: return "LA_OK";
@@ -219,11 +245,13 @@ const char* lightning_attn_status_string(int status) {
 int lightning_attn_device_status(int* status, int reset) {
   if (!status) return LA_ERR_NULL;
   int v = 0;
-  if (cudaMemcpyFromSymbol(&v, la::g_status, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, la::g_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
   *status = v ? LA_ERR_TIMEOUT : LA_OK;
   if (reset) {
     const int zero = 0;
-    if (cudaMemcpyToSymbol(la::g_status, &zero, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
+    e = cudaMemcpyToSymbol(la::g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
   }
   return LA_OK;
 }

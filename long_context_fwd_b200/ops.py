@@ -31,6 +31,7 @@ SIGNATURES = {
     "lightning_attn_fwd_f32": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P],
     "lightning_attn_decode": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P],
     "lightning_attn_status_string": [_I],
+    "lightning_attn_last_cuda_error": [],
     "lightning_attn_device_status": [_P, _I],
 }
 
@@ -39,7 +40,10 @@ class LightningAttnError(RuntimeError):
     """A C-ABI call returned a non-zero status."""
 
     def __init__(self, fn: str, code: int):
-        super().__init__(f"{fn} failed: {status_string(code)} (code {code})")
+        detail = ""
+        if code == 5:
+            detail = f" [{lib().lightning_attn_last_cuda_error().decode()}]"
+        super().__init__(f"{fn} failed: {status_string(code)} (code {code}){detail}")
         self.code = code
 
 
@@ -60,7 +64,8 @@ def lib():
             for name, argtypes in SIGNATURES.items():
                 fn = getattr(L, name)
                 fn.argtypes = argtypes
-                fn.restype = ctypes.c_char_p if name == "lightning_attn_status_string" else _I
+                fn.restype = (ctypes.c_char_p if name in ("lightning_attn_status_string",
+                                                          "lightning_attn_last_cuda_error") else _I)
             _lib = L
     return _lib
 
