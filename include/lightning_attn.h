@@ -94,6 +94,39 @@ int lightning_attn_fwd_ex(const void* q, const void* k, const void* v,
                           int D, int E, int chunk, void* stream);
 
 /*
+ * Allocation-free variant of lightning_attn_fwd (the pages have no counterpart:
+ * this is an interface for callers, not part of the method).
+ *
+ * Some callers cannot allocate device memory on the call path: processes whose
+ * device memory is carved up once at start-up by their own allocator (which a
+ * cudaMallocAsync inside the library would bypass), and latency-critical
+ * serving loops where an allocation may block, trim a memory pool or fail under
+ * fragmentation.  This entry point performs no allocation and no free.  When a
+ * sequence split is used it keeps the chunk-scan scratch in one fixed device
+ * array of LA_NOALLOC_SCRATCH_BYTES bytes, compiled into the library; every
+ * device that loads the library holds that array until the process exits.
+ *
+ *   q, k, v, slopes, out, B, H, N, D, E, stream: as lightning_attn_fwd.
+ *   chunk: as lightning_attn_fwd_ex (0 = automatic).
+ * Scratch needed when the sequences are split: 256-byte-rounded
+ * (2 B H + 1) * 4 bytes of counters plus B H * 128 KiB of chunk states.  A call
+ * that would need more than LA_NOALLOC_SCRATCH_BYTES returns LA_ERR_WORKSPACE
+ * before launching anything.  With chunk = 0 the split is only used when B*H
+ * is below the SM count, which stays within the limit on a 148-SM B200.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ * capture.  All calls on a device share the one array and it keeps the last
+ * call's contents (the counters are cleared with cudaMemsetAsync on `stream`
+ * at every call): calls whose kernels overlap on the GPU -- e.g. issued on
+ * different streams without ordering between them -- race on it and must be
+ * serialised by the caller.
+ */
+#define LA_NOALLOC_SCRATCH_BYTES (20u * 1024u * 1024u)
+int lightning_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                               const float* slopes, float* out, int B, int H,
+                               int N, int D, int E, int chunk, void* stream);
+
+/*
  * Prefill with fp32 inputs and output (same operation and layout as
  * lightning_attn_fwd, all tensors fp32).  D, E in {64, 128}.  CUDA-core fp32
  * arithmetic, for callers that need fp32-class accuracy.

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "lightning_attn.h"
 #include "sm100_ptx.cuh"
 #include "tmap.h"
@@ -150,6 +152,96 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   return rc;
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free prefill: the chunk-scan scratch lives in a fixed device array.
+// ---------------------------------------------------------------------------
+// The array's name is only a host-side stand-in in host code; its device
+// address is fetched per device with cudaGetSymbolAddress (first call on each
+// device) and cached.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch_ptr(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return LA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return LA_OK;
+}
+
+int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const float* slopes,
+                          float* out, int B, int H, int N, int D, int E, int chunk,
+                          void* stream_ptr) {
+  if (!q || !k || !v || !slopes || !out) return LA_ERR_NULL;
+  if (!dims_ok(B, H, N, D, E)) return LA_ERR_SHAPE;
+  if (D != 128 || E != 128) return LA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(slopes))
+    return LA_ERR_ALIGN;
+  if (chunk < 0 || (chunk % 128) != 0) return LA_ERR_SHAPE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  const int nseq = B * H;
+  const int sms = sm_count();
+  const int nblk = (N + 127) / 128;
+  int L = chunk > 0 ? chunk : auto_chunk(nseq, N, sms);
+  if (L >= nblk * 128) L = nblk * 128;
+  const int nchunks = (N + L - 1) / L;
+  const long long total = static_cast<long long>(nseq) * nchunks;
+  if (total >= (1ll << 31)) return LA_ERR_SHAPE;
+  const size_t ctrl = ((static_cast<size_t>(nseq) * 2 + 1) * sizeof(int) + 255) / 256 * 256;
+  const size_t bytes = ctrl + static_cast<size_t>(nseq) * 2 * 128 * 128 * sizeof(float);
+  if (nchunks > 1 && bytes > LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_WORKSPACE;
+
+  CUtensorMap tq, tk, tv, to;
+  if (!la::make_tmap_3d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
+      !la::make_tmap_3d(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
+      !la::make_tmap_3d(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
+      !la::make_tmap_3d(&to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, N, nseq, 32, 128))
+    return LA_ERR_CUDA;
+
+  la::fwd::Params p{};
+  p.slopes = slopes;
+  p.status = status_word();
+  if (!p.status) return LA_ERR_CUDA;
+  p.H = H;
+  p.N = N;
+  p.nseq = nseq;
+  p.L = L;
+  p.nchunks = nchunks;
+  p.total = static_cast<int>(total);
+  p.wait_limit_ns = kWaitLimitNs;
+  if (nchunks > 1) {
+    void* scratch = nullptr;
+    const int rc = noalloc_scratch_ptr(&scratch);
+    if (rc != LA_OK) return rc;
+    // the array keeps the previous call's contents: the ticket and the flags
+    // must start at zero (the chunk states are always written before read)
+    const cudaError_t e = cudaMemsetAsync(scratch, 0, ctrl, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    p.ticket = static_cast<int*>(scratch);
+    p.flags = p.ticket + 1;
+    p.prefix = reinterpret_cast<float*>(static_cast<char*>(scratch) + ctrl);
+  }
+  const cudaError_t attr =
+      cudaFuncSetAttribute(la::fwd::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           la::fwd::SMEM_BYTES);
+  if (attr != cudaSuccess) return cuda_fail(attr);
+  const int grid = static_cast<int>(total < sms ? total : sms);
+  la::fwd::fwd_bf16_kernel<<<grid, la::fwd::THREADS, la::fwd::SMEM_BYTES, stream>>>(tq, tk, tv, to,
+                                                                                  p);
+  return launch_status();
+}
+
 template <int D, int E>
 int launch_f32(const float* q, const float* k, const float* v, const float* slopes, float* out,
                int B, int H, int N, cudaStream_t stream) {
@@ -185,6 +277,12 @@ int lightning_attn_fwd_ex(const void* q, const void* k, const void* v, const flo
                           int N, int D, int E, int chunk, void* stream) {
   return fwd_bf16_impl(q, k, v, slopes, init_state, final_state, out, B, H, N, D, E, chunk,
                        stream);
+}
+
+int lightning_attn_fwd_noalloc(const void* q, const void* k, const void* v, const float* slopes,
+                               float* out, int B, int H, int N, int D, int E, int chunk,
+                               void* stream) {
+  return fwd_bf16_noalloc_impl(q, k, v, slopes, out, B, H, N, D, E, chunk, stream);
 }
 
 int lightning_attn_fwd_f32(const float* q, const float* k, const float* v, const float* slopes,

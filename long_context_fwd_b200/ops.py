@@ -28,6 +28,7 @@ _P, _I = ctypes.c_void_p, ctypes.c_int
 SIGNATURES = {
     "lightning_attn_fwd": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P],
     "lightning_attn_fwd_ex": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P],
+    "lightning_attn_fwd_noalloc": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P],
     "lightning_attn_fwd_f32": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P],
     "lightning_attn_decode": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P],
     "lightning_attn_status_string": [_I],
@@ -124,6 +125,30 @@ def fwd(q, k, v, slopes, out=None, *, init_state=None, final_state=None, chunk: 
             None if final_state is None else final_state.data_ptr(),
             out.data_ptr(), B, H, N, D, E, int(chunk), _stream_handle(stream))
         _check("lightning_attn_fwd_ex", rc)
+    return out
+
+
+def fwd_noalloc(q, k, v, slopes, out=None, *, chunk: int = 0, stream=None) -> torch.Tensor:
+    """Prefill through the allocation-free entry point (scratch in a fixed device array).
+
+    For callers that must not allocate device memory on the call path; see
+    lightning_attn_fwd_noalloc in include/lightning_attn.h for the limit and
+    the rule that overlapping calls on one device race on the shared scratch.
+    `out` should be passed preallocated by such callers.
+    """
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    _need(q, "q", torch.bfloat16, (B, H, N, D))
+    _need(k, "k", torch.bfloat16, (B, H, N, D))
+    _need(v, "v", torch.bfloat16, (B, H, N, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    if out is None:
+        out = torch.empty((B, H, N, E), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, H, N, E))
+    rc = lib().lightning_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                          slopes.data_ptr(), out.data_ptr(), B, H, N, D, E,
+                                          int(chunk), _stream_handle(stream))
+    _check("lightning_attn_fwd_noalloc", rc)
     return out
 
 
