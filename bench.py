@@ -52,11 +52,12 @@ def parse():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="prefill_b4h64n32768d128")
+    ap.add_argument("--workload", default="prefill_b4h64n32768d128",
+                    help="prefill workload timed for the headline value (profiling uses the 8K one)")
     ap.add_argument("--chunk", type=int, default=0, help="prefill chunk length (0 = automatic)")
     ap.add_argument("--decode-steps", type=int, default=1024)
-    ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the end-to-end leg")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="0 skips the CPU baseline")
     ap.add_argument("--no-decode", action="store_true")
     return ap.parse_args()
 
@@ -65,28 +66,34 @@ def parse():
 # distributed plumbing
 # ----------------------------------------------------------------------------
 class Dist:
+    """One process per GPU (torchrun env vars); NCCL on GPUs, gloo for CPU tests."""
+
     def __init__(self):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.backend = None
 
-    def init(self, backend):
+    def init(self, backend, timeout_s: int = 300):
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
             self.pg = dist
+            self.backend = backend
 
     def barrier(self):
         if self.pg:
             self.pg.barrier()
 
     def max(self, x: float) -> float:
+        """Max over ranks (device timings are reported as the slowest rank's)."""
         if not self.pg:
             return x
         import torch
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dev = "cpu" if self.backend == "gloo" else "cuda"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
@@ -182,6 +189,11 @@ def bench_prefill(args, dist, w, dev):
     status = ops.device_status(reset=True)
     res = {"total_ms": dist.max(total_ms), "launch_ms": dist.max(launch_ms),
            "window": (t_host0, t_host1), "status": status}
+    if args.e2e_steps <= 0:
+        res["e2e_ms"], res["h2d"], res["d2h"] = None, 0, 0
+        del q, k, v, out
+        torch.cuda.empty_cache()
+        return res
     # end to end through host buffers: pinned inputs in, result out, every step
     hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -278,6 +290,12 @@ def cpu_baseline(w, seconds: float):
                       f"({dt:.1f} s)"}
 
 
+def job_throughput(world: int, units_per_rank: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput: every rank processes its own units each step; the
+    step takes as long as the slowest rank."""
+    return world * units_per_rank / (ms_per_step_max / 1e3)
+
+
 def main_ours(args):
     import torch
     from long_context_fwd_b200 import inputs as I
@@ -295,7 +313,7 @@ def main_ours(args):
     clocks = sampler.stop()
     tokens_step = w.B * w.N
     ms_step = pre["total_ms"] / args.steps
-    value = dist.world * tokens_step / (ms_step / 1e3)
+    value = job_throughput(dist.world, tokens_step, ms_step)
     bytes_launch = w.B * w.H * w.N * BYTES_PER_TOKEN_HEAD
     achieved = bytes_launch / (pre["launch_ms"] / 1e3) / 1e9
     flops_launch = w.B * w.H * w.N * (4 * w.D * w.E + 2 * BLK * (w.D + w.E))
@@ -324,9 +342,10 @@ def main_ours(args):
                      "tensor_peak_tflops": bf16},
         "gpu_launches": args.steps,
         "device_status": pre["status"],
-        "e2e": {"value": dist.world * tokens_step / (pre["e2e_ms"] / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"],
-                "ms_per_step": pre["e2e_ms"]},
+        "e2e": None if pre["e2e_ms"] is None else {
+            "value": job_throughput(dist.world, tokens_step, pre["e2e_ms"]), "unit": "tokens/s",
+            "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"],
+            "ms_per_step": pre["e2e_ms"]},
         "clocks": clocks,
     }
     if dec:
@@ -336,7 +355,7 @@ def main_ours(args):
                           "gpu_launches": dec["steps"], "state_finite": dec["finite"],
                           "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                                        "frac": gbs / hbm, "bytes_per_launch": dec["bytes"]}}
-    if dist.rank == 0 and dist.world == 1:
+    if dist.rank == 0 and dist.world == 1 and args.cpu_seconds > 0:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if dist.rank == 0:
         print(json.dumps(line), flush=True)

@@ -149,6 +149,24 @@ int lightning_attn_decode(const void* q, const void* k, const void* v,
                           int B, int H, int D, int E, void* stream);
 
 /*
+ * Fault-injection hook for testing the bounded device-side waits (an interface
+ * for tests; the pages have no counterpart).  Runs the chunked bf16 prefill
+ * (D = E = 128, chunk a multiple of 128 with N > chunk) but hands out work
+ * starting at chunk 1: chunk 0 is never processed, so every chunk-1 item waits
+ * on a publication flag that nothing sets.  Each device-side wait of this
+ * launch gives up after wait_limit_ms milliseconds (1..10000); the kernel then
+ * records LA_ERR_TIMEOUT in the device status word (read it with
+ * lightning_attn_device_status), waits for its own copies and MMAs in flight,
+ * releases its tensor memory and returns.  `out` is left unspecified.  No
+ * fault, trap or unbounded wait is involved; the context stays usable.
+ */
+int lightning_attn_fault_test_scan_stall(const void* q, const void* k,
+                                         const void* v, const float* slopes,
+                                         float* out, int B, int H, int N,
+                                         int chunk, unsigned int wait_limit_ms,
+                                         void* stream);
+
+/*
  * Text of the CUDA runtime error behind the calling thread's most recent
  * LA_ERR_CUDA (static string, never NULL; "no error" before any).
  */

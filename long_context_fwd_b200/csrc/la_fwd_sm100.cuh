@@ -56,6 +56,8 @@ constexpr int BLK = 128;  // tokens per block (= MMA M)
 constexpr int HD = 128;   // D = E = 128
 constexpr int X_THREADS = 256;
 constexpr int Y_THREADS = 128;
+constexpr int X_WARPS = X_THREADS / 32;
+constexpr int Y_WARPS = Y_THREADS / 32;
 constexpr int X_WARP0 = 0;
 constexpr int Y_WARP0 = 8;
 constexpr int PRODUCER_WARP = 12;
@@ -251,10 +253,17 @@ __device__ __forceinline__ bool cwait(const Ctx& c, const Params& p, int id, uin
   return ok;
 }
 
+// One arrival per warp once every lane has reached this point (the barriers
+// the compute groups signal count warps, not threads).
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if (lane_id() == 0) mbar_arrive(bar);
+}
+
 // Synchronises the threads of one compute group through an mbarrier
 // (bounded, unlike bar.sync, so a failed wait elsewhere cannot hang the group).
 __device__ __forceinline__ bool gsync(const Ctx& c, const Params& p, int id, uint32_t& n) {
-  mbar_arrive(&c.bar[id]);
+  warp_arrive(&c.bar[id]);
   return cwait(c, p, id, n++ & 1u);
 }
 
@@ -460,7 +469,7 @@ __device__ void group_x(const Ctx& c, const Params& p) {
     const uint32_t ws = w_it & 1u;
     if (!cwait(c, p, B_WF + ws, (w_it >> 1) & 1u)) break;
     const int w = static_cast<int>(c.misc[1 + ws]);
-    mbar_arrive(&c.bar[B_WE + ws]);
+    warp_arrive(&c.bar[B_WE + ws]);
     ++w_it;
     if (w >= p.total) break;
     const Item it = decode_item(p, w);
@@ -480,7 +489,7 @@ __device__ void group_x(const Ctx& c, const Params& p) {
         const float f = jc < it.Lc ? expf(-lam * static_cast<float>(it.Lc - 1 - jc)) : 0.f;
         scale_row(c.sbase + OFF_K + ks * TILE + hf * PLANE + r * 128u, r, f);
         fence_proxy_async_smem();
-        mbar_arrive(&c.bar[B_KT + ks]);
+        warp_arrive(&c.bar[B_KT + ks]);
         if (t == 0) LA_TRACE_EVENT(22, k_it);
         ++k_it;
       }
@@ -529,7 +538,7 @@ __device__ void group_x(const Ctx& c, const Params& p) {
           qv[4 * ch + 2] = scale_bf16x2(x.z, fq);
           qv[4 * ch + 3] = scale_bf16x2(x.w, fq);
         }
-        mbar_arrive(&c.bar[B_QE + qs]);
+        warp_arrive(&c.bar[B_QE + qs]);
         tmem_st32(t_s + 32u, qv);
       }
       // gamma^(len-1-r) K (0 past len) in place
@@ -538,7 +547,7 @@ __device__ void group_x(const Ctx& c, const Params& p) {
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&c.bar[B_READY]);
+      warp_arrive(&c.bar[B_READY]);
       if (t == 0) LA_TRACE_EVENT(10, g);
       ++q_it;
       ++k_it;
@@ -615,12 +624,12 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     const uint32_t ws = w_it & 1u;
     if (!cwait(c, p, B_WF + ws, (w_it >> 1) & 1u)) break;
     const int w = static_cast<int>(c.misc[1 + ws]);
-    mbar_arrive(&c.bar[B_WE + ws]);
+    warp_arrive(&c.bar[B_WE + ws]);
     ++w_it;
     if (w >= p.total) break;
     const Item it = decode_item(p, w);
     const float lam = p.slopes[it.seq % p.H];
-    mbar_arrive(&c.bar[B_KV_FREE]);  // done with the previous item's state
+    warp_arrive(&c.bar[B_KV_FREE]);  // done with the previous item's state
     if (leader) LA_TRACE_EVENT(15, w_it);
     if (it.phase1) v_it += it.nb;
 
@@ -690,7 +699,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     fence_proxy_async_smem();
     tmem_wait_st();
     tc_fence_before();
-    mbar_arrive(&c.bar[B_KVB_READY]);
+    warp_arrive(&c.bar[B_KVB_READY]);
     if (leader) LA_TRACE_EVENT(20, w_it);
 
     bool ok = true;
@@ -723,7 +732,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
           fence_proxy_async_smem();
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(&c.bar[B_KVB_READY]);
+          warp_arrive(&c.bar[B_KVB_READY]);
         }
         if (leader) LA_TRACE_EVENT(12, g);
       }
@@ -752,7 +761,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
       tmem_ld32(t_o + 96u, o1);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&c.bar[B_O_EMPTY]);
+      warp_arrive(&c.bar[B_O_EMPTY]);
       if (leader) bulk_wait_group_read<0>();
       if (!gsync(c, p, B_YSYNC, ys_n)) { ok = false; break; }
       store_row_f32(vtile + r * 128u, r, o0);
@@ -793,7 +802,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&c.bar[B_QF + i], 1);
-      mbar_init(&c.bar[B_QE + i], X_THREADS);
+      mbar_init(&c.bar[B_QE + i], X_WARPS);
       mbar_init(&c.bar[B_KF + i], 1);
       mbar_init(&c.bar[B_KE + i], 1);
       mbar_init(&c.bar[B_VF + i], 1);
@@ -801,18 +810,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&c.bar[B_SF + i], 1);
       mbar_init(&c.bar[B_SE + i], 1);
       mbar_init(&c.bar[B_WF + i], 1);
-      mbar_init(&c.bar[B_WE + i], 1 + X_THREADS + Y_THREADS);
-      mbar_init(&c.bar[B_KT + i], X_THREADS);
+      mbar_init(&c.bar[B_WE + i], 1 + X_WARPS + Y_WARPS);
+      mbar_init(&c.bar[B_KT + i], X_WARPS);
     }
-    mbar_init(&c.bar[B_READY], X_THREADS);
-    mbar_init(&c.bar[B_KVB_READY], Y_THREADS);
+    mbar_init(&c.bar[B_READY], X_WARPS);
+    mbar_init(&c.bar[B_KVB_READY], Y_WARPS);
     mbar_init(&c.bar[B_KVO_DONE], 1);
     mbar_init(&c.bar[B_O_FULL], 1);
-    mbar_init(&c.bar[B_O_EMPTY], Y_THREADS);
+    mbar_init(&c.bar[B_O_EMPTY], Y_WARPS);
     mbar_init(&c.bar[B_AGG_FULL], 1);
-    mbar_init(&c.bar[B_KV_FREE], Y_THREADS);
-    mbar_init(&c.bar[B_XSYNC], X_THREADS);
-    mbar_init(&c.bar[B_YSYNC], Y_THREADS);
+    mbar_init(&c.bar[B_KV_FREE], Y_WARPS);
+    mbar_init(&c.bar[B_XSYNC], X_WARPS);
+    mbar_init(&c.bar[B_YSYNC], Y_WARPS);
     mbar_init(&c.bar[B_DRAIN], 1);
     c.misc[3] = 0;
     fence_mbar_init();

@@ -77,7 +77,8 @@ int auto_chunk(int nseq, int N, int sms) {
 
 int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slopes,
                   const float* init_state, float* final_state, float* out, int B, int H, int N,
-                  int D, int E, int chunk, void* stream_ptr) {
+                  int D, int E, int chunk, void* stream_ptr, int first_chunk = 0,
+                  unsigned long long wait_limit_ns = kWaitLimitNs) {
   if (!q || !k || !v || !slopes || !out) return LA_ERR_NULL;
   if (!dims_ok(B, H, N, D, E)) return LA_ERR_SHAPE;
   if (D != 128 || E != 128) return LA_ERR_UNSUPPORTED;
@@ -114,7 +115,8 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   p.L = L;
   p.nchunks = nchunks;
   p.total = static_cast<int>(total);
-  p.wait_limit_ns = kWaitLimitNs;
+  p.ticket_base = first_chunk * nseq;
+  p.wait_limit_ns = wait_limit_ns;
 
   void* scratch = nullptr;
   if (nchunks > 1) {
@@ -277,6 +279,15 @@ int lightning_attn_fwd_ex(const void* q, const void* k, const void* v, const flo
                           int N, int D, int E, int chunk, void* stream) {
   return fwd_bf16_impl(q, k, v, slopes, init_state, final_state, out, B, H, N, D, E, chunk,
                        stream);
+}
+
+int lightning_attn_fault_test_scan_stall(const void* q, const void* k, const void* v,
+                                         const float* slopes, float* out, int B, int H, int N,
+                                         int chunk, unsigned int wait_limit_ms, void* stream) {
+  if (chunk <= 0 || N <= chunk) return LA_ERR_SHAPE;  // needs at least two chunks
+  if (wait_limit_ms == 0 || wait_limit_ms > 10000) return LA_ERR_SHAPE;
+  return fwd_bf16_impl(q, k, v, slopes, nullptr, nullptr, out, B, H, N, 128, 128, chunk, stream,
+                       /*first_chunk=*/1, 1000000ull * wait_limit_ms);
 }
 
 int lightning_attn_fwd_noalloc(const void* q, const void* k, const void* v, const float* slopes,

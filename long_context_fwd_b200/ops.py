@@ -30,6 +30,7 @@ SIGNATURES = {
     "lightning_attn_fwd_ex": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P],
     "lightning_attn_fwd_noalloc": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P],
     "lightning_attn_fwd_f32": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P],
+    "lightning_attn_fault_test_scan_stall": [_P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_uint, _P],
     "lightning_attn_decode": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P],
     "lightning_attn_status_string": [_I],
     "lightning_attn_last_cuda_error": [],
@@ -186,6 +187,22 @@ def decode(q, k, v, state, slopes, out=None, *, stream=None) -> torch.Tensor:
                                      _stream_handle(stream))
     _check("lightning_attn_decode", rc)
     return out
+
+
+def fault_test_scan_stall(q, k, v, slopes, out, *, chunk: int, wait_limit_ms: int,
+                          stream=None) -> None:
+    """Runs the prefill with chunk 0 never processed (see the C header): every
+    chunk-1 item waits on a flag nothing sets until its bounded wait gives up."""
+    B, H, N, D = q.shape
+    _need(q, "q", torch.bfloat16, (B, H, N, 128))
+    _need(k, "k", torch.bfloat16, (B, H, N, 128))
+    _need(v, "v", torch.bfloat16, (B, H, N, 128))
+    _need(slopes, "slopes", torch.float32, (H,))
+    _need(out, "out", torch.float32, (B, H, N, 128))
+    rc = lib().lightning_attn_fault_test_scan_stall(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), slopes.data_ptr(), out.data_ptr(), B, H, N,
+        int(chunk), int(wait_limit_ms), _stream_handle(stream))
+    _check("lightning_attn_fault_test_scan_stall", rc)
 
 
 def device_status(reset: bool = True) -> int:

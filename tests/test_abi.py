@@ -94,3 +94,18 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ops.fwd(x, x, x, torch.zeros(1))
+
+
+def test_fault_hook_validation(lib):
+    f = lib.lightning_attn_fault_test_scan_stall
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1024, 0, 100, None) == LA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 256, 256, 100, None) == LA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1024, 256, 0, None) == LA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1024, 256, 20000, None) == LA_ERR_SHAPE
+
+
+def test_noalloc_rejects_oversized_scratch_on_host(lib):
+    # 200 sequences in 128-token chunks need 25 MiB of chunk states: rejected
+    # before any launch.
+    f = lib.lightning_attn_fwd_noalloc
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 200, 1024, 128, 128, 128, None) == 7
