@@ -78,14 +78,23 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
 constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_KV = 384;
 
+// Phase 1 reads only K and V.  It lays a 3-deep ring of (K, V) pairs over the
+// Q/K/V ring memory (pair slot p = [p * 2 TILE, +2 TILE): K then V), so three
+// blocks are in flight instead of two.  Pair slot p overlaps phase-2 ring p
+// (0: Q, 1: K, 2: V); the producer hands memory over between the two layouts.
+constexpr int P1_SLOTS = 3;
+__host__ __device__ constexpr uint32_t p1_base(uint32_t slot) { return OFF_Q + slot * 2u * TILE; }
+
 enum BarId : int {
   B_QF = 0, B_QE = 2, B_KF = 4, B_KE = 6, B_VF = 8, B_VE = 10,
   B_SF = 12, B_SE = 14,
   B_READY = 16, B_KVB_READY, B_KVO_DONE, B_O_FULL, B_O_EMPTY, B_AGG_FULL, B_KV_FREE,
   B_WF = 24, B_WE = 26,
   B_XSYNC = 28, B_YSYNC = 29, B_DRAIN = 30,
-  B_KT = 32,  // phase 1: decayed K tile ready, one per K slot (2)
-  B_COUNT = 34
+  B_P1F = 32,  // phase 1: K/V pair loaded, one per pair slot (3)
+  B_P1E = 35,  // phase 1: pair slot free again (3)
+  B_KT = 38,   // phase 1: decayed K tile of a pair slot ready (3)
+  B_COUNT = 41
 };
 
 struct Params {
@@ -307,6 +316,22 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
     drain_ring(B_KF, k_it);
     drain_ring(B_VF, v_it);
   };
+  uint32_t p1_it = 0;  // phase-1 pair loads issued
+  // Waits until the phase-2 ring overlapping pair slot `slot` has released its
+  // last two tiles (their phases have completed, so these waits do not alias).
+  auto ring_released = [&](uint32_t slot) -> bool {
+    const int e = slot == 0 ? B_QE : slot == 1 ? B_KE : B_VE;
+    const uint32_t n = slot == 0 ? q_it : slot == 1 ? k_it : v_it;
+    for (uint32_t j = n >= 2 ? n - 2 : 0; j < n; ++j)
+      if (!wait_bar(c, p, e + (j & 1u), (j >> 1) & 1u)) return false;
+    return true;
+  };
+  // Waits until every phase-1 pair issued so far has been consumed.
+  auto pairs_released = [&]() -> bool {
+    for (uint32_t j = p1_it >= P1_SLOTS ? p1_it - P1_SLOTS : 0; j < p1_it; ++j)
+      if (!wait_bar(c, p, B_P1E + (j % P1_SLOTS), (j / P1_SLOTS) & 1u)) return false;
+    return true;
+  };
   for (;;) {
     const int w = next_work(p, static_next);
     const uint32_t ws = w_it & 1u;
@@ -319,10 +344,21 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
     bool ok = true;
     if (it.phase1) {
       for (int b = 0; b < it.nb && ok; ++b) {
+        const uint32_t slot = p1_it % P1_SLOTS, use = p1_it / P1_SLOTS;
+        if (b < P1_SLOTS) ok = ring_released(slot);  // first use in this item
+        if (ok && use >= 1) ok = wait_bar(c, p, B_P1E + slot, (use - 1) & 1u);
+        if (!ok) break;
         const int row = it.t0 + b * BLK;
-        ok = load(B_KF, B_KE, OFF_K, k_it, tk, row, it.seq, pol_last) &&
-             load(B_VF, B_VE, OFF_V, v_it, tv, row, it.seq, pol_last);
+        uint8_t* dst = c.sm + p1_base(slot);
+        uint64_t* full = &c.bar[B_P1F + slot];
+        mbar_arrive_expect_tx(full, 2 * TILE);
+        tma_load_3d(dst, tk, full, 0, row, it.seq, pol_last);
+        tma_load_3d(dst + PLANE, tk, full, 64, row, it.seq, pol_last);
+        tma_load_3d(dst + TILE, tv, full, 0, row, it.seq, pol_last);
+        tma_load_3d(dst + TILE + PLANE, tv, full, 64, row, it.seq, pol_last);
+        ++p1_it;
       }
+      if (ok) ok = pairs_released();  // phase-2 tiles reuse that memory
     }
     for (int n = 0; n < it.nb && ok; ++n) {
       const int row = it.t0 + n * BLK;
@@ -332,6 +368,8 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
     }
     if (!ok) break;
   }
+  for (uint32_t j = p1_it >= P1_SLOTS ? p1_it - P1_SLOTS : 0; j < p1_it; ++j)
+    mbar_wait(&c.bar[B_P1F + (j % P1_SLOTS)], (j / P1_SLOTS) & 1u, p.wait_limit_ns);
   drain();
 }
 
@@ -345,8 +383,7 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
   const uint32_t sbase = c.sbase;
   const uint32_t kvb = sbase + OFF_KVB;
   uint32_t q_it = 0, k_it = 0, v_it = 0, w_it = 0, gb = 0;
-  uint32_t ready_n = 0, kvb_n = 0, kvfree_n = 0;
-  uint32_t kt_n[2] = {0, 0};
+  uint32_t ready_n = 0, kvb_n = 0, kvfree_n = 0, p1_it = 0;
 
   // S/P buffer (gidx & 1) <- Q K^T for global phase-2 block gidx.
   auto issue_S = [&](uint32_t qi, uint32_t ki, uint32_t gidx) -> bool {
@@ -378,19 +415,16 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
     if (!wait_bar(c, p, B_KV_FREE, kvfree_n++ & 1u)) return;
     if (it.phase1) {
       for (int b = 0; b < it.nb; ++b) {
-        const uint32_t ks = k_it & 1u, vs = v_it & 1u;
-        if (!wait_bar(c, p, B_KT + ks, kt_n[ks]++ & 1u)) return;
-        if (!wait_bar(c, p, B_VF + vs, (v_it >> 1) & 1u)) return;
+        const uint32_t slot = p1_it % P1_SLOTS;
+        if (!wait_bar(c, p, B_KT + slot, (p1_it / P1_SLOTS) & 1u)) return;
         tc_fence_after();
-        const uint32_t ka = sbase + OFF_K + ks * TILE, va = sbase + OFF_V + vs * TILE;
+        const uint32_t ka = sbase + p1_base(slot), va = ka + TILE;
 #pragma unroll
         for (uint32_t kk = 0; kk < 8; ++kk)
           mma_ss(c.tmem + TM_KV, sdesc_sw128(ka + kk * 2048u, PLANE, 1024),
                  sdesc_sw128(va + kk * 2048u, PLANE, 1024), ID_AMN, (b > 0) || (kk > 0));
-        mma_commit(&c.bar[B_KE + ks]);
-        mma_commit(&c.bar[B_VE + vs]);
-        ++k_it;
-        ++v_it;
+        mma_commit(&c.bar[B_P1E + slot]);
+        ++p1_it;
       }
       mma_commit(&c.bar[B_AGG_FULL]);
       LA_TRACE_EVENT(21, w_it);
@@ -464,7 +498,7 @@ __device__ void group_x(const Ctx& c, const Params& p) {
   const uint32_t hf = warp >> 2;
   const uint32_t lane_base = ((warp & 3u) * 32u) << 16;
   const uint32_t gtab = c.sbase + OFF_GTAB;
-  uint32_t q_it = 0, k_it = 0, w_it = 0, gb = 0, xs_n = 0;
+  uint32_t q_it = 0, k_it = 0, w_it = 0, gb = 0, xs_n = 0, p1_it = 0;
   for (;;) {
     const uint32_t ws = w_it & 1u;
     if (!cwait(c, p, B_WF + ws, (w_it >> 1) & 1u)) break;
@@ -483,15 +517,15 @@ __device__ void group_x(const Ctx& c, const Params& p) {
     bool ok = true;
     if (it.phase1) {  // K rows decayed to the chunk end: gamma^(Lc-1-j)
       for (int b = 0; b < it.nb && ok; ++b) {
-        const uint32_t ks = k_it & 1u;
-        if (!cwait(c, p, B_KF + ks, (k_it >> 1) & 1u)) { ok = false; break; }
+        const uint32_t slot = p1_it % P1_SLOTS;
+        if (!cwait(c, p, B_P1F + slot, (p1_it / P1_SLOTS) & 1u)) { ok = false; break; }
         const int jc = b * BLK + static_cast<int>(r);
         const float f = jc < it.Lc ? expf(-lam * static_cast<float>(it.Lc - 1 - jc)) : 0.f;
-        scale_row(c.sbase + OFF_K + ks * TILE + hf * PLANE + r * 128u, r, f);
+        scale_row(c.sbase + p1_base(slot) + hf * PLANE + r * 128u, r, f);
         fence_proxy_async_smem();
-        warp_arrive(&c.bar[B_KT + ks]);
-        if (t == 0) LA_TRACE_EVENT(22, k_it);
-        ++k_it;
+        warp_arrive(&c.bar[B_KT + slot]);
+        if (t == 0) LA_TRACE_EVENT(22, p1_it);
+        ++p1_it;
       }
     }
     for (int n = 0; n < it.nb && ok; ++n) {
@@ -631,7 +665,6 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     const float lam = p.slopes[it.seq % p.H];
     warp_arrive(&c.bar[B_KV_FREE]);  // done with the previous item's state
     if (leader) LA_TRACE_EVENT(15, w_it);
-    if (it.phase1) v_it += it.nb;
 
     // ---- entering state; publication of this chunk's inclusive state ----
     const float* scan_src = nullptr;  // previous chunk's state (scan layout)
@@ -811,6 +844,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&c.bar[B_SE + i], 1);
       mbar_init(&c.bar[B_WF + i], 1);
       mbar_init(&c.bar[B_WE + i], 1 + X_WARPS + Y_WARPS);
+    }
+    for (int i = 0; i < P1_SLOTS; ++i) {
+      mbar_init(&c.bar[B_P1F + i], 1);
+      mbar_init(&c.bar[B_P1E + i], 1);
       mbar_init(&c.bar[B_KT + i], X_WARPS);
     }
     mbar_init(&c.bar[B_READY], X_WARPS);
