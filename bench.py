@@ -36,6 +36,39 @@ BYTES_PER_TOKEN_HEAD = 2 * 128 + 2 * 128 + 2 * 128 + 4 * 128  # q, k, v bf16 in 
 BLK = 128  # tokens per block in the prefill kernel
 
 
+KERNEL_SOURCES = ("long_context_fwd_b200/csrc/la_fwd_sm100.cuh",
+                  "long_context_fwd_b200/csrc/sm100_ptx.cuh")
+PROFILE = os.path.join(ROOT, "profiles", "prefill_bf16_tcgen05.md")
+
+
+def kernel_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload) -> "float | None":
+    """DRAM bytes per launch of the prefill kernel from the committed ncu summary,
+    scaled to `workload` by (b, h, token) units; None unless the summary was
+    taken on the current kernel source."""
+    try:
+        fields = {}
+        with open(PROFILE) as f:
+            for line in f:
+                if line.startswith("- ") and ":" in line:
+                    k, v = line[2:].split(":", 1)
+                    fields[k.strip()] = v.strip().strip("`")
+        if fields.get("kernel_sha") != kernel_hash():
+            return None
+        per_unit = float(fields["dram_bytes_per_launch"]) / float(fields["token_heads_per_launch"])
+        return per_unit * workload.B * workload.H * workload.N
+    except Exception:
+        return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -335,7 +368,7 @@ def main_ours(args):
                    "parallelism": f"replicas x{dist.world} (independent (b,h) problems, no collective)",
                    "l2": "no flush: each step streams 10.7 GB, far larger than the 126 MB L2"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None,
+                     "frac": achieved / hbm, "traffic": measured_traffic(w),
                      "peak_source": f"{peak_src} copy bandwidth",
                      "bytes_per_launch": bytes_launch, "kernel_ms": pre["launch_ms"],
                      "tensor_tflops": flops_launch / (pre["launch_ms"] / 1e3) / 1e12,

@@ -68,8 +68,13 @@ PREFILL_1M = Workload("prefill_b1h64n1048576d128", 1, 64, 1048576, 128, 128, "bf
 DECODE = Workload("decode_b256h64d128_1024steps", 256, 64, 1, 128, 128, "bf16", steps=1024,
                   kind="decode", index=4)
 
+# Profiling case: one wave of whole sequences (148 = the B200 SM count), the
+# unsplit code path of the 32K workload at 1.5 GB instead of 10.7 GB.
+PROFILE_148x8K = Workload("profile_prefill_b1h148n8192d128", 1, 148, 8192, 128, 128, "bf16",
+                          index=5)
+
 WORKLOADS = {w.name: w for w in (TINY_F32, TINY_F32_NODECAY, PREFILL_8K, PREFILL_32K,
-                                 PREFILL_1M, DECODE)}
+                                 PREFILL_1M, DECODE, PROFILE_148x8K)}
 
 
 def alibi_slopes(H: int) -> np.ndarray:
