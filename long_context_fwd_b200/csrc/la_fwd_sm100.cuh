@@ -107,18 +107,23 @@ struct Params {
   int* status;                // sticky error word
   int H, N, nseq, L, nchunks, total;
   int ticket_base;            // first ticket handed out (0 except in fault-injection runs)
+  int balanced;               // static balanced split with final-state hand-off (no phase 1)
   unsigned long long wait_limit_ns;
 };
 
 struct Item {
   int seq, chunk, t0, Lc, nb;
-  bool phase1;
+  bool phase1;   // local state first, published before the outputs (parallel scan)
+  bool publish;  // final state published after the outputs (balanced split)
+  bool enter;    // starts from a published state: prefix[enter_slot] once flags[enter_slot] == enter_val
+  bool last;     // ends its sequence (final state goes to the caller)
+  int enter_slot, enter_val, pub_slot, pub_val;
 };
 
 // Optional event trace (compiled only with -DLA_TRACE): %globaltimer stamps of
 // each role's pipeline events for the first few CTAs, for timeline analysis.
 #ifdef LA_TRACE
-constexpr int TRACE_CTAS = 4, TRACE_EVENTS = 24, TRACE_SLOTS = 256;
+constexpr int TRACE_CTAS = 4, TRACE_EVENTS = 28, TRACE_SLOTS = 256;
 __device__ unsigned long long* g_trace;
 __device__ __forceinline__ void trace_event(int ev, uint32_t idx) {
   if (g_trace && blockIdx.x < TRACE_CTAS && idx < TRACE_SLOTS)
@@ -129,6 +134,8 @@ __device__ __forceinline__ void trace_event(int ev, uint32_t idx) {
 #define LA_TRACE_EVENT(ev, idx) ((void)0)
 #endif
 
+// Ticket w of a chunked or unchunked run: chunk-major order, so every chunk of
+// a sequence is handed out after its predecessor.
 __device__ __forceinline__ Item decode_item(const Params& p, int w) {
   Item it;
   it.chunk = w / p.nseq;
@@ -137,7 +144,87 @@ __device__ __forceinline__ Item decode_item(const Params& p, int w) {
   it.Lc = min(p.L, p.N - it.t0);
   it.nb = (it.Lc + BLK - 1) / BLK;
   it.phase1 = it.chunk + 1 < p.nchunks;
+  it.publish = false;
+  it.enter = it.chunk > 0;
+  it.last = it.chunk + 1 == p.nchunks;
+  it.enter_slot = it.seq * 2 + ((it.chunk - 1) & 1);
+  it.enter_val = it.chunk;
+  it.pub_slot = it.seq * 2 + (it.chunk & 1);
+  it.pub_val = it.chunk + 1;
   return it;
+}
+
+// Balanced split (at least as many sequences as CTAs): CTA j owns blocks
+// [j*T/G, (j+1)*T/G) of the concatenation of all sequences' 128-token blocks
+// (T blocks, G CTAs), at least one whole sequence's worth.  So at most one
+// sequence crosses each CTA boundary: CTA j computes that sequence's first part
+// FIRST and publishes its final state in slot j; CTA j+1 computes the rest LAST,
+// starting from slot j, which by then has long been written.  Item k of this CTA:
+// the first part (if any), the whole sequences in order, then the rest of the
+// sequence that CTA j-1 began (if any).
+// The CTA's split, computed once at launch into misc[4..9]: head sequence and
+// its length in blocks (0: none), first whole sequence and their count, tail
+// sequence and its first block (0: none).
+__device__ void balanced_split(const Params& p, volatile uint32_t* m) {
+  const int64_t nblk = (p.N + BLK - 1) / BLK;
+  const int64_t T = nblk * p.nseq, G = gridDim.x, j = blockIdx.x;
+  const int64_t b0 = T * j / G, b1 = T * (j + 1) / G;
+  const int64_t s_first = b0 / nblk, s_last = (b1 - 1) / nblk;
+  const int64_t tail_b0 = b0 - s_first * nblk;          // > 0: continues CTA j-1's sequence
+  const int64_t head_len = b1 < (s_last + 1) * nblk ? b1 - s_last * nblk : 0;
+  const int64_t full0 = s_first + (tail_b0 ? 1 : 0), full1 = s_last + (head_len ? 0 : 1);
+  m[4] = static_cast<uint32_t>(s_last);
+  m[5] = static_cast<uint32_t>(head_len);
+  m[6] = static_cast<uint32_t>(full0);
+  m[7] = static_cast<uint32_t>(full1 > full0 ? full1 - full0 : 0);
+  m[8] = static_cast<uint32_t>(s_first);
+  m[9] = static_cast<uint32_t>(tail_b0);
+}
+
+__device__ __forceinline__ bool balanced_item(const Params& p, const volatile uint32_t* m, int k,
+                                              Item& it) {
+  const int nblk = (p.N + BLK - 1) / BLK;
+  const int head_len = static_cast<int>(m[5]), nfull = static_cast<int>(m[7]);
+  const int tail_b0 = static_cast<int>(m[9]);
+  int seq, blk0 = 0, blk1 = nblk;
+  it.phase1 = false;
+  it.publish = it.enter = false;
+  it.enter_slot = static_cast<int>(blockIdx.x) - 1;
+  it.pub_slot = static_cast<int>(blockIdx.x);
+  it.enter_val = it.pub_val = 1;
+  int i = k;
+  if (head_len && i == 0) {
+    seq = static_cast<int>(m[4]);
+    blk1 = head_len;
+    it.publish = true;
+  } else {
+    if (head_len) --i;
+    if (i < nfull) {
+      seq = static_cast<int>(m[6]) + i;
+    } else if (tail_b0 && i == nfull) {
+      seq = static_cast<int>(m[8]);
+      blk0 = tail_b0;
+      it.enter = true;
+    } else {
+      return false;
+    }
+  }
+  it.seq = seq;
+  it.chunk = it.enter ? 1 : 0;
+  it.t0 = blk0 * BLK;
+  it.Lc = min(blk1 * BLK, p.N) - it.t0;
+  it.nb = blk1 - blk0;
+  it.last = !it.publish;
+  return true;
+}
+
+// Work item for work index w; false once this CTA has no more.
+__device__ __forceinline__ bool get_item(const Params& p, const volatile uint32_t* m, int w,
+                                         Item& it) {
+  if (p.balanced) return balanced_item(p, m, w, it);
+  if (w >= p.total) return false;
+  it = decode_item(p, w);
+  return true;
 }
 
 __device__ __forceinline__ void st_release_gpu(int* ptr, int v) {
@@ -234,7 +321,8 @@ struct Ctx {
   uint8_t* sm;
   uint32_t sbase;           // shared-space address of sm
   uint64_t* bar;
-  volatile uint32_t* misc;  // [0] TMEM base, [1..2] work slots, [3] abort
+  volatile uint32_t* misc;  // [0] TMEM base, [1..2] work slots, [3] abort,
+                            // [4..9] balanced split of this CTA
   uint32_t tmem;
 };
 
@@ -276,12 +364,12 @@ __device__ __forceinline__ bool gsync(const Ctx& c, const Params& p, int id, uin
   return cwait(c, p, id, n++ & 1u);
 }
 
-// Next work item: dynamic ticket for chunked runs, static stride otherwise.
-__device__ __forceinline__ int next_work(const Params& p, int& static_next) {
+// Next work index: this CTA's item count in a balanced split, a dynamic ticket
+// for chunked runs, a static stride otherwise (n counts this CTA's items).
+__device__ __forceinline__ int next_work(const Params& p, int& n) {
+  if (p.balanced) return n++;
   if (p.nchunks > 1) return p.ticket_base + atomicAdd(p.ticket, 1);
-  const int w = static_next;
-  static_next += gridDim.x;
-  return w;
+  return blockIdx.x + gridDim.x * n++;
 }
 
 // ---------------------------------------------------------------------------
@@ -292,7 +380,7 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
   const uint64_t pol_first = policy_evict_first();
   const uint64_t pol_last = policy_evict_last();
   uint32_t q_it = 0, k_it = 0, v_it = 0, w_it = 0;
-  int static_next = blockIdx.x;
+  int n_items = 0;
   auto load = [&](int ring_f, int ring_e, uint32_t off, uint32_t& it, const CUtensorMap* tm,
                   int row, int seq, uint64_t pol) -> bool {
     const uint32_t s = it & 1u;
@@ -333,14 +421,14 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
     return true;
   };
   for (;;) {
-    const int w = next_work(p, static_next);
+    const int w = next_work(p, n_items);
     const uint32_t ws = w_it & 1u;
     if (w_it >= 2 && !wait_bar(c, p, B_WE + ws, ((w_it >> 1) - 1) & 1u)) break;
     c.misc[1 + ws] = static_cast<uint32_t>(w);
     mbar_arrive(&c.bar[B_WF + ws]);
     ++w_it;
-    if (w >= p.total) break;
-    const Item it = decode_item(p, w);
+    Item it;
+    if (!get_item(p, c.misc, w, it)) break;
     bool ok = true;
     if (it.phase1) {
       for (int b = 0; b < it.nb && ok; ++b) {
@@ -410,8 +498,8 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
     const int w = static_cast<int>(c.misc[1 + ws]);
     mbar_arrive(&c.bar[B_WE + ws]);
     ++w_it;
-    if (w >= p.total) return;
-    const Item it = decode_item(p, w);
+    Item it;
+    if (!get_item(p, c.misc, w, it)) return;
     if (!wait_bar(c, p, B_KV_FREE, kvfree_n++ & 1u)) return;
     if (it.phase1) {
       for (int b = 0; b < it.nb; ++b) {
@@ -505,8 +593,8 @@ __device__ void group_x(const Ctx& c, const Params& p) {
     const int w = static_cast<int>(c.misc[1 + ws]);
     warp_arrive(&c.bar[B_WE + ws]);
     ++w_it;
-    if (w >= p.total) break;
-    const Item it = decode_item(p, w);
+    Item it;
+    if (!get_item(p, c.misc, w, it)) break;
     const float lam = p.slopes[it.seq % p.H];
 
     // decay table: gtab[u] = gamma^(127-u) for u <= 127, 0 above (the causal mask)
@@ -660,8 +748,8 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     const int w = static_cast<int>(c.misc[1 + ws]);
     warp_arrive(&c.bar[B_WE + ws]);
     ++w_it;
-    if (w >= p.total) break;
-    const Item it = decode_item(p, w);
+    Item it;
+    if (!get_item(p, c.misc, w, it)) break;
     const float lam = p.slopes[it.seq % p.H];
     warp_arrive(&c.bar[B_KV_FREE]);  // done with the previous item's state
     if (leader) LA_TRACE_EVENT(15, w_it);
@@ -669,13 +757,12 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     // ---- entering state; publication of this chunk's inclusive state ----
     const float* scan_src = nullptr;  // previous chunk's state (scan layout)
     const float* init_src = nullptr;  // caller's initial state (row layout)
-    if (it.chunk > 0) {
-      const int slot = (it.chunk - 1) & 1;
+    if (it.enter) {
       if (leader) {
-        const int* flag = p.flags + it.seq * 2 + slot;
+        const int* flag = p.flags + it.enter_slot;
         const uint64_t t0 = globaltimer_ns();
         uint32_t spins = 0;
-        while (ld_acquire_gpu(flag) != it.chunk) {
+        while (ld_acquire_gpu(flag) != it.enter_val) {
           if ((++spins & 15u) == 0 && (aborted(c) || globaltimer_ns() - t0 > p.wait_limit_ns)) {
             fail(c, p, 2);
             break;
@@ -683,7 +770,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         }
       }
       if (!gsync(c, p, B_YSYNC, ys_n)) break;
-      scan_src = p.prefix + (static_cast<int64_t>(it.seq) * 2 + slot) * (HD * HD);
+      scan_src = p.prefix + static_cast<int64_t>(it.enter_slot) * (HD * HD);
     } else if (p.init_state) {
       init_src = p.init_state + static_cast<int64_t>(it.seq) * (HD * HD) + row_off;
     }
@@ -694,7 +781,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     {
       const float gL = expf(-lam * static_cast<float>(it.Lc));
       const float g0 = expf(-lam * static_cast<float>(min(BLK, it.Lc)));
-      float* pub = p.prefix + (static_cast<int64_t>(it.seq) * 2 + (it.chunk & 1)) * (HD * HD);
+      float* pub = p.prefix + static_cast<int64_t>(it.pub_slot) * (HD * HD);
 #pragma unroll 1
       for (uint32_t q = 0; q < 4; ++q) {
         uint32_t prev[32];
@@ -725,7 +812,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
       if (!gsync(c, p, B_YSYNC, ys_n)) break;
       if (leader) {
         __threadfence();
-        st_release_gpu(p.flags + it.seq * 2 + (it.chunk & 1), it.chunk + 1);
+        st_release_gpu(p.flags + it.pub_slot, it.pub_val);
       }
     }
     if (leader) LA_TRACE_EVENT(19, w_it);
@@ -735,6 +822,14 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     warp_arrive(&c.bar[B_KVB_READY]);
     if (leader) LA_TRACE_EVENT(20, w_it);
 
+    // where the state after the item's last block goes: the caller's final
+    // state (row layout) or a balanced split's hand-over slot (scan layout)
+    float* const fin_dst =
+        it.last && p.final_state ? p.final_state + static_cast<int64_t>(it.seq) * (HD * HD) + row_off
+                                 : nullptr;
+    float* const pub_dst = it.publish ? p.prefix + static_cast<int64_t>(it.pub_slot) * (HD * HD) : nullptr;
+    int* const pub_flag = it.publish ? p.flags + it.pub_slot : nullptr;
+    const int pub_val = it.pub_val;
     bool ok = true;
     for (int n = 0; n < it.nb && ok; ++n) {
       const uint32_t g = gb;
@@ -747,7 +842,8 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         const bool more = n + 1 < it.nb;
         const float gnext =
             more ? expf(-lam * static_cast<float>(min(BLK, it.Lc - (n + 1) * BLK))) : 1.f;
-        const bool fin = !more && p.final_state && it.chunk + 1 == p.nchunks;
+        const bool fin = !more && fin_dst != nullptr;
+        const bool pub = !more && pub_dst != nullptr;
 #pragma unroll 1
         for (uint32_t q = 0; q < 4; ++q) {
           uint32_t kv[32];
@@ -757,8 +853,9 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
             store_half_bf16(kvb_row(q), r, q & 1u, kv, 1.f);
             tmem_st32_scaled(t_kv + 32u * q, kv, gnext);
           } else if (fin) {
-            st_global32(p.final_state + static_cast<int64_t>(it.seq) * (HD * HD) + row_off + 32 * q,
-                        kv);
+            st_global32(fin_dst + 32 * q, kv);
+          } else if (pub) {
+            st_scan32(pub_dst, r, q >> 1, q & 1u, kv);
           }
         }
         if (more) {
@@ -766,6 +863,14 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
           tmem_wait_st();
           tc_fence_before();
           warp_arrive(&c.bar[B_KVB_READY]);
+        } else if (pub) {
+          // the state goes to the CTA that continues this sequence: the
+          // group's stores are ordered before the leader's fence and release
+          if (!gsync(c, p, B_YSYNC, ys_n)) { ok = false; break; }
+          if (leader) {
+            __threadfence();
+            st_release_gpu(pub_flag, pub_val);
+          }
         }
         if (leader) LA_TRACE_EVENT(12, g);
       }
@@ -789,13 +894,16 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         tma_store_3d(to, vtile_g, 0, row, it.seq, pol_out);
         tma_store_3d(to, vtile_g + PLANE, 32, row, it.seq, pol_out);
         bulk_commit_group();
+        LA_TRACE_EVENT(23, g);
       }
       tmem_ld32(t_o + 64u, o0);
       tmem_ld32(t_o + 96u, o1);
       tmem_wait_ld();
       tc_fence_before();
       warp_arrive(&c.bar[B_O_EMPTY]);
+      if (leader) LA_TRACE_EVENT(24, g);
       if (leader) bulk_wait_group_read<0>();
+      if (leader) LA_TRACE_EVENT(25, g);
       if (!gsync(c, p, B_YSYNC, ys_n)) { ok = false; break; }
       store_row_f32(vtile + r * 128u, r, o0);
       store_row_f32(vtile + PLANE + r * 128u, r, o1);
@@ -805,6 +913,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         tma_store_3d(to, vtile_g, 64, row, it.seq, pol_out);
         tma_store_3d(to, vtile_g + PLANE, 96, row, it.seq, pol_out);
         bulk_commit_group();
+        LA_TRACE_EVENT(26, g);
         bulk_wait_group_read<0>();
         mbar_arrive(&c.bar[B_VE + vs]);
       }
@@ -861,6 +970,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&c.bar[B_YSYNC], Y_WARPS);
     mbar_init(&c.bar[B_DRAIN], 1);
     c.misc[3] = 0;
+    if (p.balanced) balanced_split(p, c.misc);
     fence_mbar_init();
   }
   if (warp == MMA_WARP) {

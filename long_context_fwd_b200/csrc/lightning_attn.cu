@@ -61,18 +61,74 @@ int sm_count() {
   return n;
 }
 
-// Chunk length for the sequence split.  Whole sequences when there are at
-// least as many (b, h) problems as SMs (splitting costs a local-state pass and a
-// scan step per chunk); otherwise chunks of 2048-8192 tokens (measured sweet
-// spot on B200) so that the work items cover a few waves of SMs.
-int auto_chunk(int nseq, int N, int sms) {
+// How the (b, h) sequences become work items for the persistent grid.
+//  * Fewer sequences than SMs: a parallel scan over chunks of 2048-8192 tokens
+//    (measured sweet spot on B200) so that the items cover a few waves of SMs.
+//    Every chunk but the last first computes its local state (an extra pass
+//    over its K and V) and publishes its inclusive state, then its outputs.
+//  * At least as many sequences as SMs: a balanced split.  Each CTA gets the
+//    same number of 128-token blocks of the concatenated sequences; a sequence
+//    that crosses a CTA boundary is handed over through its final state (no
+//    extra pass), and the two CTAs order their work so that the hand-over is
+//    not waited for.  Without this, 256 sequences on 148 SMs would take two
+//    full waves with 40 SMs idle in the second.
+//  * An explicit chunk length shorter than N always selects the parallel scan.
+struct Plan {
+  int L = 0, nchunks = 1, balanced = 0, grid = 0;
+  long long total = 0;
+  size_t ctrl = 0, bytes = 0;  // scratch: ticket + flags, then 64 KiB chunk states
+};
+
+Plan make_plan(int nseq, int N, int sms, int chunk) {
+  Plan pl;
   const int nblk = (N + 127) / 128;
-  if (nseq >= sms || nblk <= 8) return nblk * 128;
-  const int want_chunks = (4 * sms + nseq - 1) / nseq;
-  int L = ((N + want_chunks - 1) / want_chunks + 127) / 128 * 128;
-  if (L < 2048) L = 2048;
-  if (L > 8192) L = 8192;
-  return L;
+  const size_t state_bytes = 128 * 128 * sizeof(float);
+  auto round256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  if (chunk == 0 && nseq >= sms) {
+    pl.balanced = 1;
+    pl.L = nblk * 128;
+    pl.grid = sms;
+    if (nseq % sms != 0) {  // some sequence crosses a CTA boundary
+      pl.ctrl = round256((static_cast<size_t>(sms) + 1) * sizeof(int));
+      pl.bytes = pl.ctrl + static_cast<size_t>(sms) * state_bytes;
+    }
+    return pl;
+  }
+  int L = chunk;
+  if (L == 0) {
+    L = nblk * 128;
+    if (nblk > 8) {
+      const int want_chunks = (4 * sms + nseq - 1) / nseq;
+      L = ((N + want_chunks - 1) / want_chunks + 127) / 128 * 128;
+      if (L < 2048) L = 2048;
+      if (L > 8192) L = 8192;
+    }
+  }
+  if (L > nblk * 128) L = nblk * 128;
+  pl.L = L;
+  pl.nchunks = (N + L - 1) / L;
+  pl.total = static_cast<long long>(nseq) * pl.nchunks;
+  pl.grid = static_cast<int>(pl.total < sms ? pl.total : sms);
+  if (pl.nchunks > 1) {
+    pl.ctrl = round256((static_cast<size_t>(nseq) * 2 + 1) * sizeof(int));
+    pl.bytes = pl.ctrl + static_cast<size_t>(nseq) * 2 * state_bytes;
+  }
+  return pl;
+}
+
+// Fills the launch parameters that depend on the plan.
+void apply_plan(const Plan& pl, int nseq, la::fwd::Params& p) {
+  p.nseq = nseq;
+  p.L = pl.L;
+  p.nchunks = pl.nchunks;
+  p.total = static_cast<int>(pl.total);
+  p.balanced = pl.balanced;
+}
+
+void set_scratch(const Plan& pl, void* scratch, la::fwd::Params& p) {
+  p.ticket = static_cast<int*>(scratch);
+  p.flags = p.ticket + 1;
+  p.prefix = reinterpret_cast<float*>(static_cast<char*>(scratch) + pl.ctrl);
 }
 
 int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slopes,
@@ -89,12 +145,8 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   const int nseq = B * H;
   const int sms = sm_count();
-  const int nblk = (N + 127) / 128;
-  int L = chunk > 0 ? chunk : auto_chunk(nseq, N, sms);
-  if (L >= nblk * 128) L = nblk * 128;
-  const int nchunks = (N + L - 1) / L;
-  const long long total = static_cast<long long>(nseq) * nchunks;
-  if (total >= (1ll << 31)) return LA_ERR_SHAPE;
+  const Plan pl = make_plan(nseq, N, sms, chunk);
+  if (pl.total >= (1ll << 31)) return LA_ERR_SHAPE;
 
   CUtensorMap tq, tk, tv, to;
   if (!la::make_tmap_3d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
@@ -111,27 +163,20 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   if (!p.status) return LA_ERR_CUDA;
   p.H = H;
   p.N = N;
-  p.nseq = nseq;
-  p.L = L;
-  p.nchunks = nchunks;
-  p.total = static_cast<int>(total);
+  apply_plan(pl, nseq, p);
   p.ticket_base = first_chunk * nseq;
   p.wait_limit_ns = wait_limit_ns;
 
   void* scratch = nullptr;
-  if (nchunks > 1) {
-    const size_t ctrl = ((static_cast<size_t>(nseq) * 2 + 1) * sizeof(int) + 255) / 256 * 256;
-    const size_t bytes = ctrl + static_cast<size_t>(nseq) * 2 * 128 * 128 * sizeof(float);
-    cudaError_t e = cudaMallocAsync(&scratch, bytes, stream);
+  if (pl.bytes) {
+    cudaError_t e = cudaMallocAsync(&scratch, pl.bytes, stream);
     if (e != cudaSuccess) return cuda_fail(e);
-    e = cudaMemsetAsync(scratch, 0, ctrl, stream);
+    e = cudaMemsetAsync(scratch, 0, pl.ctrl, stream);
     if (e != cudaSuccess) {
       cudaFreeAsync(scratch, stream);
       return cuda_fail(e);
     }
-    p.ticket = static_cast<int*>(scratch);
-    p.flags = p.ticket + 1;
-    p.prefix = reinterpret_cast<float*>(static_cast<char*>(scratch) + ctrl);
+    set_scratch(pl, scratch, p);
   }
 
   // set on every call: the attribute belongs to the current device's context
@@ -142,9 +187,8 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   if (attr != cudaSuccess) {
     rc = cuda_fail(attr);
   } else {
-    const int grid = static_cast<int>(total < sms ? total : sms);
-    la::fwd::fwd_bf16_kernel<<<grid, la::fwd::THREADS, la::fwd::SMEM_BYTES, stream>>>(tq, tk, tv,
-                                                                                    to, p);
+    la::fwd::fwd_bf16_kernel<<<pl.grid, la::fwd::THREADS, la::fwd::SMEM_BYTES, stream>>>(
+        tq, tk, tv, to, p);
     rc = launch_status();
   }
   if (scratch) {
@@ -194,15 +238,16 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   const int nseq = B * H;
   const int sms = sm_count();
-  const int nblk = (N + 127) / 128;
-  int L = chunk > 0 ? chunk : auto_chunk(nseq, N, sms);
-  if (L >= nblk * 128) L = nblk * 128;
-  const int nchunks = (N + L - 1) / L;
-  const long long total = static_cast<long long>(nseq) * nchunks;
-  if (total >= (1ll << 31)) return LA_ERR_SHAPE;
-  const size_t ctrl = ((static_cast<size_t>(nseq) * 2 + 1) * sizeof(int) + 255) / 256 * 256;
-  const size_t bytes = ctrl + static_cast<size_t>(nseq) * 2 * 128 * 128 * sizeof(float);
-  if (nchunks > 1 && bytes > LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_WORKSPACE;
+  Plan pl = make_plan(nseq, N, sms, chunk);
+  if (pl.balanced && pl.bytes > LA_NOALLOC_SCRATCH_BYTES) {
+    // a GPU with so many SMs that the hand-over states do not fit: whole sequences
+    pl = Plan{};
+    pl.L = (N + 127) / 128 * 128;
+    pl.total = nseq;
+    pl.grid = nseq < sms ? nseq : sms;
+  }
+  if (pl.total >= (1ll << 31)) return LA_ERR_SHAPE;
+  if (pl.bytes > LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_WORKSPACE;
 
   CUtensorMap tq, tk, tv, to;
   if (!la::make_tmap_3d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
@@ -217,30 +262,24 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
   if (!p.status) return LA_ERR_CUDA;
   p.H = H;
   p.N = N;
-  p.nseq = nseq;
-  p.L = L;
-  p.nchunks = nchunks;
-  p.total = static_cast<int>(total);
+  apply_plan(pl, nseq, p);
   p.wait_limit_ns = kWaitLimitNs;
-  if (nchunks > 1) {
+  if (pl.bytes) {
     void* scratch = nullptr;
     const int rc = noalloc_scratch_ptr(&scratch);
     if (rc != LA_OK) return rc;
     // the array keeps the previous call's contents: the ticket and the flags
     // must start at zero (the chunk states are always written before read)
-    const cudaError_t e = cudaMemsetAsync(scratch, 0, ctrl, stream);
+    const cudaError_t e = cudaMemsetAsync(scratch, 0, pl.ctrl, stream);
     if (e != cudaSuccess) return cuda_fail(e);
-    p.ticket = static_cast<int*>(scratch);
-    p.flags = p.ticket + 1;
-    p.prefix = reinterpret_cast<float*>(static_cast<char*>(scratch) + ctrl);
+    set_scratch(pl, scratch, p);
   }
   const cudaError_t attr =
       cudaFuncSetAttribute(la::fwd::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            la::fwd::SMEM_BYTES);
   if (attr != cudaSuccess) return cuda_fail(attr);
-  const int grid = static_cast<int>(total < sms ? total : sms);
-  la::fwd::fwd_bf16_kernel<<<grid, la::fwd::THREADS, la::fwd::SMEM_BYTES, stream>>>(tq, tk, tv, to,
-                                                                                  p);
+  la::fwd::fwd_bf16_kernel<<<pl.grid, la::fwd::THREADS, la::fwd::SMEM_BYTES, stream>>>(tq, tk, tv,
+                                                                                     to, p);
   return launch_status();
 }
 

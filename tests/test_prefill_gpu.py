@@ -105,6 +105,46 @@ def test_bf16_initial_and_final_state(chunk):
     assert rel(fin.cpu().numpy(), sref) <= TOL_BF16
 
 
+# At least as many (b, h) sequences as the B200's 148 SMs.  With the automatic
+# chunk length the kernel splits the blocks evenly over the SMs and hands the
+# sequences that cross a CTA boundary over through their final state; an
+# explicit chunk length selects the parallel scan instead.  Ragged ends included.
+MANY_SEQ_CASES = [
+    # B, H, N, chunk
+    (1, 150, 2500, 0),
+    (2, 80, 1100, 0),
+    (1, 149, 1025, 0),
+    (1, 296, 300, 0),
+    (2, 80, 1100, 256),
+]
+
+
+@pytest.mark.parametrize("B,H,N,chunk", MANY_SEQ_CASES)
+def test_bf16_many_sequences(B, H, N, chunk):
+    sl = I.alibi_slopes(H)
+    sl[::7] = 0.0
+    q, k, v, _ = _bf16_case(B, H, N, [0.0] * H, seed=20 + H)
+    got = _run(q, k, v, sl, chunk=chunk)
+    ref = oracle.recurrent(q, k, v, sl)
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+
+
+def test_bf16_many_sequences_initial_and_final_state():
+    B, H, N = 1, 150, 900
+    sl = I.alibi_slopes(H)
+    sl[3::5] = 0.0
+    q, k, v, _ = _bf16_case(B, H, N, [0.0] * H, seed=31)
+    s0 = (np.random.default_rng(7).standard_normal((B, H, 128, 128)) * 0.02).astype(np.float32)
+    fin = torch.zeros((B, H, 128, 128), dtype=torch.float32, device=DEV)
+    got = _run(q, k, v, sl, init_state=f32_to_dev(s0, DEV), final_state=fin)
+    ref, sref = oracle.recurrent(q, k, v, sl, s0=s0.astype(np.float64), return_state=True)
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+    assert rel(fin.cpu().numpy(), sref) <= TOL_BF16
+    assert worst_head(fin.cpu().numpy(), sref) <= TOL_BF16
+
+
 def test_bf16_prefill_then_decode_continues_sequence():
     B, H, N, T = 2, 2, 700, 6
     w = I.Workload("handoff", B, H, N + T, 128, 128, "bf16", index=140)

@@ -34,6 +34,10 @@ def test_noalloc_matches_allocating_entry_point_twice(chunk):
     # B*H = 6 is below the SM count, so the sequences are split into chunks and
     # the chunk scan runs through the fixed scratch array.
     cases = [_case(1, 2, 3, 3000, [0.9, 0.05, 0.0]), _case(2, 1, 6, 2500, [0.3] * 5 + [0.0])]
+    if chunk == 0:
+        # more sequences than SMs: the balanced split hands sequences over
+        # between CTAs through the same fixed array
+        cases.append(_case(3, 1, 150, 1100, [0.5, 0.02, 0.0] * 50))
     for q, k, v, sl in cases:
         out_na = torch.full(q.shape[:3] + (128,), float("nan"), dtype=torch.float32, device=DEV)
         ops.fwd_noalloc(q, k, v, sl, out_na, chunk=chunk)
