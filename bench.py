@@ -37,7 +37,8 @@ BLK = 128  # tokens per block in the prefill kernel
 
 
 KERNEL_SOURCES = ("long_context_fwd_b200/csrc/la_fwd_sm100.cuh",
-                  "long_context_fwd_b200/csrc/sm100_ptx.cuh")
+                  "long_context_fwd_b200/csrc/sm100_ptx.cuh",
+                  "long_context_fwd_b200/csrc/la_schedule.cuh")
 PROFILE = os.path.join(ROOT, "profiles", "prefill_bf16_tcgen05.md")
 
 

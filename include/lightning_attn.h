@@ -172,6 +172,32 @@ int lightning_attn_fault_test_scan_stall(const void* q, const void* k,
  */
 const char* lightning_attn_last_cuda_error(void);
 
+/*
+ * Scheduling diagnostic (an interface for tests; the pages have no
+ * counterpart: how work is spread over the SMs is this implementation's own).
+ * Runs on the host only, needs no GPU and touches no device memory.  For a
+ * bf16 prefill of B*H sequences of N tokens (D = E = 128) with chunk length
+ * `chunk` (0 = automatic) on a GPU with `sms` SMs, reports the plan and every
+ * work item the prefill kernel would process:
+ *   info[8]: mode (0 whole sequences / chunk scan with tickets, 1 balanced
+ *            hand-over, 2 split scan), grid size, chunk length, chunks per
+ *            sequence, split-scan first-part blocks F, split-scan output CTAs
+ *            over the first parts G2, state slots, flag words.
+ *   rec[10 * i .. 10 * i + 9] for record i: cta (-1 for ticket items), kind
+ *            (0 outputs, 1 local state only, 2 a local state chained into the
+ *            preceding kind-0 record's entering state), sequence, then for
+ *            kinds 0/1 first token and token count, for kind 2 stream blocks
+ *            [x, y); flags (1 enters from a published state, 2 publishes its
+ *            final state, 4 ends its sequence, 8 computes its local state
+ *            first); entering slot and flag value; publishing slot and value.
+ * Records are listed per CTA in processing order.  *n_rec receives the
+ * number of records; returns LA_ERR_WORKSPACE (records beyond max_rec not
+ * written) if max_rec is too small, LA_ERR_SHAPE / LA_ERR_NULL on bad
+ * arguments.
+ */
+int lightning_attn_fwd_plan(int B, int H, int N, int chunk, int sms, int* info, int* rec,
+                            int max_rec, int* n_rec);
+
 /* Human-readable name of a la_status value (static string, never NULL). */
 const char* lightning_attn_status_string(int status);
 

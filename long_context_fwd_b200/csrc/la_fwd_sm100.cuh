@@ -47,13 +47,13 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "la_schedule.cuh"
 #include "sm100_ptx.cuh"
 
 namespace la {
 namespace fwd {
 
-constexpr int BLK = 128;  // tokens per block (= MMA M)
-constexpr int HD = 128;   // D = E = 128
+// BLK (tokens per block = MMA M) and HD (D = E) come from la_schedule.cuh.
 constexpr int X_THREADS = 256;
 constexpr int Y_THREADS = 128;
 constexpr int X_WARPS = X_THREADS / 32;
@@ -73,7 +73,7 @@ constexpr uint32_t OFF_KVB = 6 * TILE;  // bf16 copy of the state (MMA B operand
 constexpr uint32_t OFF_BAR = 7 * TILE;
 constexpr uint32_t OFF_GTAB = OFF_BAR + 512;  // 256 floats: gtab[u] = gamma^(127-u), 0 for u > 127
 constexpr uint32_t OFF_MISC = OFF_GTAB + 1024;
-constexpr uint32_t SMEM_USED = OFF_MISC + 64;
+constexpr uint32_t SMEM_USED = OFF_MISC + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
 constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_KV = 384;
@@ -97,29 +97,6 @@ enum BarId : int {
   B_COUNT = 41
 };
 
-struct Params {
-  const float* slopes;        // [H]
-  float* prefix;              // [nseq][2][HD*HD] inclusive chunk states (chunked runs)
-  int* flags;                 // [nseq][2] publication flags (chunked runs), zeroed
-  int* ticket;                // work counter (chunked runs), zeroed
-  const float* init_state;    // nullable [nseq][HD*HD]
-  float* final_state;         // nullable [nseq][HD*HD]
-  int* status;                // sticky error word
-  int H, N, nseq, L, nchunks, total;
-  int ticket_base;            // first ticket handed out (0 except in fault-injection runs)
-  int balanced;               // static balanced split with final-state hand-off (no phase 1)
-  unsigned long long wait_limit_ns;
-};
-
-struct Item {
-  int seq, chunk, t0, Lc, nb;
-  bool phase1;   // local state first, published before the outputs (parallel scan)
-  bool publish;  // final state published after the outputs (balanced split)
-  bool enter;    // starts from a published state: prefix[enter_slot] once flags[enter_slot] == enter_val
-  bool last;     // ends its sequence (final state goes to the caller)
-  int enter_slot, enter_val, pub_slot, pub_val;
-};
-
 // Optional event trace (compiled only with -DLA_TRACE): %globaltimer stamps of
 // each role's pipeline events for the first few CTAs, for timeline analysis.
 #ifdef LA_TRACE
@@ -134,97 +111,10 @@ __device__ __forceinline__ void trace_event(int ev, uint32_t idx) {
 #define LA_TRACE_EVENT(ev, idx) ((void)0)
 #endif
 
-// Ticket w of a chunked or unchunked run: chunk-major order, so every chunk of
-// a sequence is handed out after its predecessor.
-__device__ __forceinline__ Item decode_item(const Params& p, int w) {
-  Item it;
-  it.chunk = w / p.nseq;
-  it.seq = w - it.chunk * p.nseq;
-  it.t0 = it.chunk * p.L;
-  it.Lc = min(p.L, p.N - it.t0);
-  it.nb = (it.Lc + BLK - 1) / BLK;
-  it.phase1 = it.chunk + 1 < p.nchunks;
-  it.publish = false;
-  it.enter = it.chunk > 0;
-  it.last = it.chunk + 1 == p.nchunks;
-  it.enter_slot = it.seq * 2 + ((it.chunk - 1) & 1);
-  it.enter_val = it.chunk;
-  it.pub_slot = it.seq * 2 + (it.chunk & 1);
-  it.pub_val = it.chunk + 1;
-  return it;
-}
-
-// Balanced split (at least as many sequences as CTAs): CTA j owns blocks
-// [j*T/G, (j+1)*T/G) of the concatenation of all sequences' 128-token blocks
-// (T blocks, G CTAs), at least one whole sequence's worth.  So at most one
-// sequence crosses each CTA boundary: CTA j computes that sequence's first part
-// FIRST and publishes its final state in slot j; CTA j+1 computes the rest LAST,
-// starting from slot j, which by then has long been written.  Item k of this CTA:
-// the first part (if any), the whole sequences in order, then the rest of the
-// sequence that CTA j-1 began (if any).
-// The CTA's split, computed once at launch into misc[4..9]: head sequence and
-// its length in blocks (0: none), first whole sequence and their count, tail
-// sequence and its first block (0: none).
-__device__ void balanced_split(const Params& p, volatile uint32_t* m) {
-  const int64_t nblk = (p.N + BLK - 1) / BLK;
-  const int64_t T = nblk * p.nseq, G = gridDim.x, j = blockIdx.x;
-  const int64_t b0 = T * j / G, b1 = T * (j + 1) / G;
-  const int64_t s_first = b0 / nblk, s_last = (b1 - 1) / nblk;
-  const int64_t tail_b0 = b0 - s_first * nblk;          // > 0: continues CTA j-1's sequence
-  const int64_t head_len = b1 < (s_last + 1) * nblk ? b1 - s_last * nblk : 0;
-  const int64_t full0 = s_first + (tail_b0 ? 1 : 0), full1 = s_last + (head_len ? 0 : 1);
-  m[4] = static_cast<uint32_t>(s_last);
-  m[5] = static_cast<uint32_t>(head_len);
-  m[6] = static_cast<uint32_t>(full0);
-  m[7] = static_cast<uint32_t>(full1 > full0 ? full1 - full0 : 0);
-  m[8] = static_cast<uint32_t>(s_first);
-  m[9] = static_cast<uint32_t>(tail_b0);
-}
-
-__device__ __forceinline__ bool balanced_item(const Params& p, const volatile uint32_t* m, int k,
-                                              Item& it) {
-  const int nblk = (p.N + BLK - 1) / BLK;
-  const int head_len = static_cast<int>(m[5]), nfull = static_cast<int>(m[7]);
-  const int tail_b0 = static_cast<int>(m[9]);
-  int seq, blk0 = 0, blk1 = nblk;
-  it.phase1 = false;
-  it.publish = it.enter = false;
-  it.enter_slot = static_cast<int>(blockIdx.x) - 1;
-  it.pub_slot = static_cast<int>(blockIdx.x);
-  it.enter_val = it.pub_val = 1;
-  int i = k;
-  if (head_len && i == 0) {
-    seq = static_cast<int>(m[4]);
-    blk1 = head_len;
-    it.publish = true;
-  } else {
-    if (head_len) --i;
-    if (i < nfull) {
-      seq = static_cast<int>(m[6]) + i;
-    } else if (tail_b0 && i == nfull) {
-      seq = static_cast<int>(m[8]);
-      blk0 = tail_b0;
-      it.enter = true;
-    } else {
-      return false;
-    }
-  }
-  it.seq = seq;
-  it.chunk = it.enter ? 1 : 0;
-  it.t0 = blk0 * BLK;
-  it.Lc = min(blk1 * BLK, p.N) - it.t0;
-  it.nb = blk1 - blk0;
-  it.last = !it.publish;
-  return true;
-}
-
-// Work item for work index w; false once this CTA has no more.
+// Work item for work index w on this CTA.
 __device__ __forceinline__ bool get_item(const Params& p, const volatile uint32_t* m, int w,
                                          Item& it) {
-  if (p.balanced) return balanced_item(p, m, w, it);
-  if (w >= p.total) return false;
-  it = decode_item(p, w);
-  return true;
+  return get_item(p, static_cast<int>(gridDim.x), static_cast<int>(blockIdx.x), m, w, it);
 }
 
 __device__ __forceinline__ void st_release_gpu(int* ptr, int v) {
@@ -322,7 +212,7 @@ struct Ctx {
   uint32_t sbase;           // shared-space address of sm
   uint64_t* bar;
   volatile uint32_t* misc;  // [0] TMEM base, [1..2] work slots, [3] abort,
-                            // [4..9] balanced split of this CTA
+                            // [4..17] this CTA's share of a static split
   uint32_t tmem;
 };
 
@@ -364,10 +254,10 @@ __device__ __forceinline__ bool gsync(const Ctx& c, const Params& p, int id, uin
   return cwait(c, p, id, n++ & 1u);
 }
 
-// Next work index: this CTA's item count in a balanced split, a dynamic ticket
+// Next work index: this CTA's item count in the static splits, a dynamic ticket
 // for chunked runs, a static stride otherwise (n counts this CTA's items).
 __device__ __forceinline__ int next_work(const Params& p, int& n) {
-  if (p.balanced) return n++;
+  if (p.mode != MODE_TICKETS) return n++;
   if (p.nchunks > 1) return p.ticket_base + atomicAdd(p.ticket, 1);
   return blockIdx.x + gridDim.x * n++;
 }
@@ -404,7 +294,8 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
     drain_ring(B_KF, k_it);
     drain_ring(B_VF, v_it);
   };
-  uint32_t p1_it = 0;  // phase-1 pair loads issued
+  uint32_t p1_it = 0;          // phase-1 pair loads issued
+  bool pairs_pending = false;  // pairs issued since the last pairs_released()
   // Waits until the phase-2 ring overlapping pair slot `slot` has released its
   // last two tiles (their phases have completed, so these waits do not alias).
   auto ring_released = [&](uint32_t slot) -> bool {
@@ -445,10 +336,14 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
         tma_load_3d(dst + TILE, tv, full, 0, row, it.seq, pol_last);
         tma_load_3d(dst + TILE + PLANE, tv, full, 64, row, it.seq, pol_last);
         ++p1_it;
+        pairs_pending = true;
       }
-      if (ok) ok = pairs_released();  // phase-2 tiles reuse that memory
     }
-    for (int n = 0; n < it.nb && ok; ++n) {
+    if (ok && it.p2 && pairs_pending) {  // phase-2 tiles reuse the pairs' memory
+      ok = pairs_released();
+      pairs_pending = false;
+    }
+    for (int n = 0; n < (it.p2 ? it.nb : 0) && ok; ++n) {
       const int row = it.t0 + n * BLK;
       ok = load(B_QF, B_QE, OFF_Q, q_it, tq, row, it.seq, pol_first) &&
            load(B_KF, B_KE, OFF_K, k_it, tk, row, it.seq, pol_first) &&
@@ -518,8 +413,8 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
       LA_TRACE_EVENT(21, w_it);
     }
     const uint32_t q0 = q_it, k0 = k_it, v0 = v_it, g0 = gb;
-    const uint32_t nb = static_cast<uint32_t>(it.nb);
-    if (!issue_S(q0, k0, g0)) return;
+    const uint32_t nb = it.p2 ? static_cast<uint32_t>(it.nb) : 0u;
+    if (nb > 0 && !issue_S(q0, k0, g0)) return;
     for (uint32_t n = 0; n < nb; ++n) {
       const uint32_t g = g0 + n;
       const uint32_t ks = (k0 + n) & 1u, vs = (v0 + n) & 1u;
@@ -616,7 +511,7 @@ __device__ void group_x(const Ctx& c, const Params& p) {
         ++p1_it;
       }
     }
-    for (int n = 0; n < it.nb && ok; ++n) {
+    for (int n = 0; n < (it.p2 ? it.nb : 0) && ok; ++n) {
       const uint32_t g = gb;
       const int len = min(BLK, it.Lc - n * BLK);
       const uint32_t qs = q_it & 1u, ks = k_it & 1u;
@@ -751,18 +646,33 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     Item it;
     if (!get_item(p, c.misc, w, it)) break;
     const float lam = p.slopes[it.seq % p.H];
+    tc_fence_before();
     warp_arrive(&c.bar[B_KV_FREE]);  // done with the previous item's state
     if (leader) LA_TRACE_EVENT(15, w_it);
 
     // ---- entering state; publication of this chunk's inclusive state ----
     const float* scan_src = nullptr;  // previous chunk's state (scan layout)
     const float* init_src = nullptr;  // caller's initial state (row layout)
+    // split scan: the entering state chains the published local states of the
+    // stream pieces [s F, X) (X = stream position of this item's first block)
+    const bool chain = it.enter && p.mode == MODE_SPLIT_SCAN;
+    const int64_t G = gridDim.x;
+    const int64_t x_lo = static_cast<int64_t>(it.seq) * p.F;
+    const int64_t x_hi = x_lo + it.t0 / BLK;
     if (it.enter) {
       if (leader) {
-        const int* flag = p.flags + it.enter_slot;
         const uint64_t t0 = globaltimer_ns();
         uint32_t spins = 0;
-        while (ld_acquire_gpu(flag) != it.enter_val) {
+        int64_t x = x_lo;
+        int slot = chain ? s1_slot(p, G, x) : it.enter_slot;
+        for (;;) {
+          if (ld_acquire_gpu(p.flags + slot) == it.enter_val) {
+            if (!chain) break;
+            x = s1_next(p, G, x);
+            if (x >= x_hi) break;
+            slot = s1_slot(p, G, x);
+            continue;
+          }
           if ((++spins & 15u) == 0 && (aborted(c) || globaltimer_ns() - t0 > p.wait_limit_ns)) {
             fail(c, p, 2);
             break;
@@ -770,10 +680,12 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         }
       }
       if (!gsync(c, p, B_YSYNC, ys_n)) break;
-      scan_src = p.prefix + static_cast<int64_t>(it.enter_slot) * (HD * HD);
-    } else if (p.init_state) {
-      init_src = p.init_state + static_cast<int64_t>(it.seq) * (HD * HD) + row_off;
+      if (!chain) scan_src = p.prefix + static_cast<int64_t>(it.enter_slot) * (HD * HD);
     }
+    // the caller's initial state enters at block 0 of a sequence (or through
+    // the chain); never into a local state
+    if (p.init_state && it.p2 && (!it.enter || chain))
+      init_src = p.init_state + static_cast<int64_t>(it.seq) * (HD * HD) + row_off;
     if (leader) LA_TRACE_EVENT(16, w_it);
     if (it.phase1 && !cwait(c, p, B_AGG_FULL, agg_n++ & 1u)) break;
     if (leader) LA_TRACE_EVENT(17, w_it);
@@ -793,6 +705,20 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) prev[i] = 0u;
         }
+        if (chain) {
+#pragma unroll 1
+          for (int64_t x = x_lo; x < x_hi;) {
+            const int64_t y = s1_next(p, G, x);
+            const float gp = expf(-lam * static_cast<float>((y - x) * BLK));
+            uint32_t part[32];
+            ld_scan32(p.prefix + static_cast<int64_t>(s1_slot(p, G, x)) * (HD * HD), r, q >> 1, q & 1u,
+                      part);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              prev[i] = __float_as_uint(fmaf(gp, __uint_as_float(prev[i]), __uint_as_float(part[i])));
+            x = y;
+          }
+        }
         if (it.phase1) {
           uint32_t agg[32];
           tmem_ld32(t_kv + 32u * q, agg);
@@ -802,8 +728,10 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
             agg[i] = __float_as_uint(fmaf(gL, __uint_as_float(prev[i]), __uint_as_float(agg[i])));
           st_scan32(pub, r, q >> 1, q & 1u, agg);
         }
-        store_half_bf16(kvb_row(q), r, q & 1u, prev, 1.f);
-        tmem_st32_scaled(t_kv + 32u * q, prev, g0);
+        if (it.p2) {
+          store_half_bf16(kvb_row(q), r, q & 1u, prev, 1.f);
+          tmem_st32_scaled(t_kv + 32u * q, prev, g0);
+        }
       }
     }
     if (leader) LA_TRACE_EVENT(18, w_it);
@@ -816,6 +744,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
       }
     }
     if (leader) LA_TRACE_EVENT(19, w_it);
+    if (!it.p2) continue;  // a local-state item has no outputs
     fence_proxy_async_smem();
     tmem_wait_st();
     tc_fence_before();
@@ -970,7 +899,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&c.bar[B_YSYNC], Y_WARPS);
     mbar_init(&c.bar[B_DRAIN], 1);
     c.misc[3] = 0;
-    if (p.balanced) balanced_split(p, c.misc);
+    if (!setup_split(p, static_cast<int>(gridDim.x), static_cast<int>(blockIdx.x), c.misc)) {
+      c.misc[4] = 0;  // cannot happen (see split_scan_setup); no work rather than wrong work
+      atomicOr(p.status, 4);
+    }
     fence_mbar_init();
   }
   if (warp == MMA_WARP) {

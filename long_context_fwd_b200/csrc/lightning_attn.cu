@@ -62,30 +62,39 @@ int sm_count() {
 }
 
 // How the (b, h) sequences become work items for the persistent grid.
-//  * Fewer sequences than SMs: a parallel scan over chunks of 2048-8192 tokens
-//    (measured sweet spot on B200) so that the items cover a few waves of SMs.
-//    Every chunk but the last first computes its local state (an extra pass
-//    over its K and V) and publishes its inclusive state, then its outputs.
-//  * At least as many sequences as SMs: a balanced split.  Each CTA gets the
-//    same number of 128-token blocks of the concatenated sequences; a sequence
-//    that crosses a CTA boundary is handed over through its final state (no
-//    extra pass), and the two CTAs order their work so that the hand-over is
-//    not waited for.  Without this, 256 sequences on 148 SMs would take two
-//    full waves with 40 SMs idle in the second.
-//  * An explicit chunk length shorter than N always selects the parallel scan.
+//  * At least as many sequences as SMs: a balanced hand-over split.  Each CTA
+//    gets the same number of 128-token blocks of the concatenated sequences; a
+//    sequence that crosses a CTA boundary is handed over through its final
+//    state (no extra pass), and the two CTAs order their work so that the
+//    hand-over is not waited for.  Without this, 256 sequences on 148 SMs
+//    would take two full waves with 40 SMs idle in the second.
+//  * Fewer sequences than SMs (at least SMs/8 of them, and more than 8 blocks
+//    each): a split scan.  Each of nseq CTAs computes the last T/G blocks of
+//    one sequence (T blocks in all, G CTAs); the other G - nseq CTAs share the
+//    first parts equally.  Every share but a sequence's first needs the state
+//    at its start, so a local-state pass over the first parts (an extra read of
+//    their K and V, shared equally by all CTAs) runs first; entering states
+//    chain the published local states.  The extra pass covers 1 - nseq/G of
+//    the tokens (57% for 64 sequences) instead of nearly all of them.
+//  * Otherwise (a handful of long sequences): a parallel scan over chunks of
+//    2048-8192 tokens (measured sweet spot on B200) handed out by an atomic
+//    ticket; every chunk but the last computes its local state first.
+//  * An explicit chunk length shorter than N always selects the chunk scan.
 struct Plan {
-  int L = 0, nchunks = 1, balanced = 0, grid = 0;
-  long long total = 0;
+  int L = 0, nchunks = 1, mode = 0, grid = 0;
+  int nblk = 0, F = 0, G2 = 0;
+  long long P = 0, total = 0;
   size_t ctrl = 0, bytes = 0;  // scratch: ticket + flags, then 64 KiB chunk states
 };
 
 Plan make_plan(int nseq, int N, int sms, int chunk) {
   Plan pl;
   const int nblk = (N + 127) / 128;
+  pl.nblk = nblk;
   const size_t state_bytes = 128 * 128 * sizeof(float);
   auto round256 = [](size_t x) { return (x + 255) / 256 * 256; };
   if (chunk == 0 && nseq >= sms) {
-    pl.balanced = 1;
+    pl.mode = la::fwd::MODE_HANDOVER;
     pl.L = nblk * 128;
     pl.grid = sms;
     if (nseq % sms != 0) {  // some sequence crosses a CTA boundary
@@ -93,6 +102,39 @@ Plan make_plan(int nseq, int N, int sms, int chunk) {
       pl.bytes = pl.ctrl + static_cast<size_t>(sms) * state_bytes;
     }
     return pl;
+  }
+  if (chunk == 0 && nblk > 8 && 8 * nseq >= sms) {
+    // tail = blocks of each sequence's last share, about T/G; of the two
+    // roundings take the one whose longest share (outputs + the local-state
+    // pass at ~0.4 of the cost per block) is shorter, and use the split only
+    // if that beats one whole sequence per SM
+    const long long T = static_cast<long long>(nseq) * nblk;
+    const long long G2 = sms - nseq;
+    double best = static_cast<double>(nblk);
+    long long best_tail = 0;
+    for (long long tail = T / sms; tail <= (T + sms - 1) / sms; ++tail) {
+      const long long F = nblk - tail, P = static_cast<long long>(nseq) * F;
+      if (tail < 1 || F < 1 || P >= (1ll << 31)) continue;
+      const long long packed = (P + G2 - 1) / G2;
+      const double span = static_cast<double>(tail > packed ? tail : packed) +
+                          0.4 * static_cast<double>((P + sms - 1) / sms);
+      if (span < best) {
+        best = span;
+        best_tail = tail;
+      }
+    }
+    if (best_tail > 0) {
+      const long long F = nblk - best_tail;
+      pl.mode = la::fwd::MODE_SPLIT_SCAN;
+      pl.L = nblk * 128;
+      pl.grid = sms;
+      pl.F = static_cast<int>(F);
+      pl.G2 = static_cast<int>(G2);
+      pl.P = static_cast<long long>(nseq) * F;
+      pl.ctrl = round256((2 * static_cast<size_t>(sms) + 1) * sizeof(int));
+      pl.bytes = pl.ctrl + 2 * static_cast<size_t>(sms) * state_bytes;
+      return pl;
+    }
   }
   int L = chunk;
   if (L == 0) {
@@ -122,7 +164,11 @@ void apply_plan(const Plan& pl, int nseq, la::fwd::Params& p) {
   p.L = pl.L;
   p.nchunks = pl.nchunks;
   p.total = static_cast<int>(pl.total);
-  p.balanced = pl.balanced;
+  p.mode = pl.mode;
+  p.nblk = pl.nblk;
+  p.F = pl.F;
+  p.G2 = pl.G2;
+  p.P = pl.P;
 }
 
 void set_scratch(const Plan& pl, void* scratch, la::fwd::Params& p) {
@@ -239,10 +285,11 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
   const int nseq = B * H;
   const int sms = sm_count();
   Plan pl = make_plan(nseq, N, sms, chunk);
-  if (pl.balanced && pl.bytes > LA_NOALLOC_SCRATCH_BYTES) {
-    // a GPU with so many SMs that the hand-over states do not fit: whole sequences
+  if (pl.mode != la::fwd::MODE_TICKETS && pl.bytes > LA_NOALLOC_SCRATCH_BYTES) {
+    // a GPU with so many SMs that the chunk states do not fit: whole sequences
     pl = Plan{};
     pl.L = (N + 127) / 128 * 128;
+    pl.nblk = (N + 127) / 128;
     pl.total = nseq;
     pl.grid = nseq < sms ? nseq : sms;
   }
@@ -366,6 +413,73 @@ int lightning_attn_decode(const void* q, const void* k, const void* v, float* st
 }
 
 const char* lightning_attn_last_cuda_error(void) { return t_last_cuda_error; }
+
+int lightning_attn_fwd_plan(int B, int H, int N, int chunk, int sms, int* info, int* rec,
+                            int max_rec, int* n_rec) {
+  if (!info || !n_rec || (max_rec > 0 && !rec)) return LA_ERR_NULL;
+  if (!dims_ok(B, H, N, 128, 128) || sms < 1 || chunk < 0 || (chunk % 128) != 0)
+    return LA_ERR_SHAPE;
+  const int nseq = B * H;
+  const Plan pl = make_plan(nseq, N, sms, chunk);
+  if (pl.total >= (1ll << 31)) return LA_ERR_SHAPE;
+  la::fwd::Params p{};
+  p.H = H;
+  p.N = N;
+  apply_plan(pl, nseq, p);
+  info[0] = pl.mode;
+  info[1] = pl.grid;
+  info[2] = pl.L;
+  info[3] = pl.nchunks;
+  info[4] = pl.F;
+  info[5] = pl.G2;
+  info[6] = static_cast<int>(pl.bytes > pl.ctrl ? (pl.bytes - pl.ctrl) / (128 * 128 * sizeof(float)) : 0);
+  info[7] = pl.ctrl ? static_cast<int>(pl.ctrl / sizeof(int)) - 1 : 0;
+  int n = 0;
+  auto put = [&](int cta, int kind, int seq, int a, int b, int flags, int es, int ev, int ps,
+                 int pv) {
+    if (n < max_rec) {
+      int* r = rec + 10 * static_cast<size_t>(n);
+      r[0] = cta; r[1] = kind; r[2] = seq; r[3] = a; r[4] = b;
+      r[5] = flags; r[6] = es; r[7] = ev; r[8] = ps; r[9] = pv;
+    }
+    ++n;
+  };
+  auto put_item = [&](int cta, const la::fwd::Item& it) {
+    const int flags = (it.enter ? 1 : 0) | (it.publish ? 2 : 0) | (it.last ? 4 : 0) |
+                      (it.phase1 ? 8 : 0);
+    put(cta, it.p2 ? 0 : 1, it.seq, it.t0, it.Lc, flags, it.enter_slot, it.enter_val, it.pub_slot,
+        it.pub_val);
+  };
+  if (pl.mode == la::fwd::MODE_TICKETS) {
+    for (int w = 0; w < static_cast<int>(pl.total); ++w) {
+      la::fwd::Item it;
+      if (!la::fwd::get_item(p, pl.grid, 0, nullptr, w, it)) break;
+      put_item(-1, it);
+    }
+  } else {
+    for (int i = 0; i < pl.grid; ++i) {
+      uint32_t m[32] = {};
+      if (!la::fwd::setup_split(p, pl.grid, i, m)) return LA_ERR_UNSUPPORTED;
+      la::fwd::Item it;
+      for (int k = 0; la::fwd::get_item(p, pl.grid, i, m, k, it); ++k) {
+        put_item(i, it);
+        if (it.enter && pl.mode == la::fwd::MODE_SPLIT_SCAN) {
+          // the pieces whose local states this entering state chains
+          const int64_t lo = static_cast<int64_t>(it.seq) * p.F, hi = lo + it.t0 / 128;
+          for (int64_t x = lo; x < hi;) {
+            const int64_t y = la::fwd::s1_next(p, pl.grid, x);
+            put(i, 2, it.seq, static_cast<int>(x), static_cast<int>(y), 0,
+                la::fwd::s1_slot(p, pl.grid, x), 1, 0, 0);
+            if (y <= x) return LA_ERR_UNSUPPORTED;
+            x = y;
+          }
+        }
+      }
+    }
+  }
+  *n_rec = n;
+  return n <= max_rec ? LA_OK : LA_ERR_WORKSPACE;
+}
 
 #ifdef LA_TRACE
 // Tracing builds only: device buffer of TRACE_CTAS x TRACE_EVENTS x TRACE_SLOTS

@@ -35,6 +35,7 @@ SIGNATURES = {
     "lightning_attn_status_string": [_I],
     "lightning_attn_last_cuda_error": [],
     "lightning_attn_device_status": [_P, _I],
+    "lightning_attn_fwd_plan": [_I, _I, _I, _I, _I, _P, _P, _I, _P],
 }
 
 
@@ -211,3 +212,25 @@ def device_status(reset: bool = True) -> int:
     _check("lightning_attn_device_status",
            lib().lightning_attn_device_status(ctypes.byref(v), 1 if reset else 0))
     return v.value
+
+
+PLAN_FIELDS = ("cta", "kind", "seq", "a", "b", "flags", "enter_slot", "enter_val", "pub_slot",
+               "pub_val")
+PLAN_INFO = ("mode", "grid", "L", "nchunks", "F", "G2", "slots", "flag_words")
+
+
+def fwd_plan(B: int, H: int, N: int, chunk: int = 0, sms: int = 148):
+    """Host-side enumeration of the prefill kernel's work items (no GPU needed):
+    returns (info dict, int32 array [n, 10] of records; see PLAN_FIELDS)."""
+    import numpy as np
+    info = (ctypes.c_int * 8)()
+    n = ctypes.c_int(0)
+    rc = lib().lightning_attn_fwd_plan(B, H, N, chunk, sms, info, None, 0, ctypes.byref(n))
+    if rc not in (0, 7):
+        _check("lightning_attn_fwd_plan", rc)
+    rec = np.zeros((max(n.value, 1), 10), np.int32)
+    _check("lightning_attn_fwd_plan",
+           lib().lightning_attn_fwd_plan(B, H, N, chunk, sms, info,
+                                         rec.ctypes.data_as(ctypes.c_void_p), n.value,
+                                         ctypes.byref(n)))
+    return dict(zip(PLAN_INFO, list(info))), rec[:n.value]

@@ -145,6 +145,47 @@ def test_bf16_many_sequences_initial_and_final_state():
     assert worst_head(fin.cpu().numpy(), sref) <= TOL_BF16
 
 
+# Fewer sequences than SMs, automatic chunking: the split scan (a shared
+# local-state pass over the first part of every sequence, then equal output
+# shares whose entering states chain the published local states).
+SPLIT_SCAN_CASES = [
+    # B, H, N
+    (1, 64, 2500),
+    (1, 20, 5000),
+    (1, 37, 1025),
+    (1, 100, 2000),
+    (2, 32, 3333),
+]
+
+
+@pytest.mark.parametrize("B,H,N", SPLIT_SCAN_CASES)
+def test_bf16_split_scan(B, H, N):
+    info, _ = ops.fwd_plan(B, H, N, 0, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert info["mode"] == 2
+    sl = I.alibi_slopes(H)
+    sl[::5] = 0.0
+    q, k, v, _ = _bf16_case(B, H, N, [0.0] * H, seed=40 + H)
+    got = _run(q, k, v, sl)
+    ref = oracle.recurrent(q, k, v, sl)
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+
+
+def test_bf16_split_scan_initial_and_final_state():
+    B, H, N = 1, 64, 3000
+    sl = I.alibi_slopes(H)
+    sl[2::6] = 0.0
+    q, k, v, _ = _bf16_case(B, H, N, [0.0] * H, seed=47)
+    s0 = (np.random.default_rng(9).standard_normal((B, H, 128, 128)) * 0.02).astype(np.float32)
+    fin = torch.zeros((B, H, 128, 128), dtype=torch.float32, device=DEV)
+    got = _run(q, k, v, sl, init_state=f32_to_dev(s0, DEV), final_state=fin)
+    ref, sref = oracle.recurrent(q, k, v, sl, s0=s0.astype(np.float64), return_state=True)
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+    assert rel(fin.cpu().numpy(), sref) <= TOL_BF16
+    assert worst_head(fin.cpu().numpy(), sref) <= TOL_BF16
+
+
 def test_bf16_prefill_then_decode_continues_sequence():
     B, H, N, T = 2, 2, 700, 6
     w = I.Workload("handoff", B, H, N + T, 128, 128, "bf16", index=140)
