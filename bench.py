@@ -54,7 +54,11 @@ def kernel_hash() -> str:
 def measured_traffic(workload) -> "float | None":
     """DRAM bytes per launch of the prefill kernel from the committed ncu summary,
     scaled to `workload` by (b, h, token) units; None unless the summary was
-    taken on the current kernel source."""
+    taken on the current kernel source.  The summary holds one capture per way
+    of splitting the work: whole sequences / the balanced hand-over
+    (`dram_bytes_per_launch`) and the split scan (`split_dram_bytes_per_launch`,
+    whose extra local-state reads scale with tokens only for the same number
+    of sequences, 64, as the 8K and 1M workloads)."""
     try:
         fields = {}
         with open(PROFILE) as f:
@@ -64,7 +68,16 @@ def measured_traffic(workload) -> "float | None":
                     fields[k.strip()] = v.strip().strip("`")
         if fields.get("kernel_sha") != kernel_hash():
             return None
-        per_unit = float(fields["dram_bytes_per_launch"]) / float(fields["token_heads_per_launch"])
+        from long_context_fwd_b200 import ops
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        mode = ops.fwd_plan(workload.B, workload.H, workload.N, 0, sms)[0]["mode"]
+        if mode == 2:
+            if workload.B * workload.H != int(fields["split_sequences"]):
+                return None
+            per_unit = (float(fields["split_dram_bytes_per_launch"]) /
+                        float(fields["split_token_heads_per_launch"]))
+        else:
+            per_unit = float(fields["dram_bytes_per_launch"]) / float(fields["token_heads_per_launch"])
         return per_unit * workload.B * workload.H * workload.N
     except Exception:
         return None
@@ -367,7 +380,8 @@ def main_ours(args):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "E": w.E,
                    "global_batch": w.B * dist.world, "seq_len": w.N, "chunk": args.chunk or "auto",
                    "parallelism": f"replicas x{dist.world} (independent (b,h) problems, no collective)",
-                   "l2": "no flush: each step streams 10.7 GB, far larger than the 126 MB L2"},
+                   "l2": f"no flush: each step streams {bytes_launch / 1e9:.2f} GB, larger than the "
+                         "126 MB L2"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": measured_traffic(w),
                      "peak_source": f"{peak_src} copy bandwidth",

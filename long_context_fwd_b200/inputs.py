@@ -73,8 +73,14 @@ DECODE = Workload("decode_b256h64d128_1024steps", 256, 64, 1, 128, 128, "bf16", 
 PROFILE_148x8K = Workload("profile_prefill_b1h148n8192d128", 1, 148, 8192, 128, 128, "bf16",
                           index=5)
 
+# Profiling case of the split scan (64 sequences on 148 SMs, the code path of
+# the 8K and 1M workloads) at 2.7 GB: the local-state pass re-reads the K and V
+# of the first 1 - 64/148 of every sequence.
+PROFILE_64x32K = Workload("profile_prefill_b1h64n32768d128", 1, 64, 32768, 128, 128, "bf16",
+                          index=7)
+
 WORKLOADS = {w.name: w for w in (TINY_F32, TINY_F32_NODECAY, PREFILL_8K, PREFILL_32K,
-                                 PREFILL_1M, DECODE, PROFILE_148x8K)}
+                                 PREFILL_1M, DECODE, PROFILE_148x8K, PROFILE_64x32K)}
 
 
 def alibi_slopes(H: int) -> np.ndarray:
