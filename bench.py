@@ -102,6 +102,8 @@ def parse():
     ap.add_argument("--workload", default="prefill_b4h64n32768d128",
                     help="prefill workload timed for the headline value (profiling uses the 8K one)")
     ap.add_argument("--chunk", type=int, default=0, help="prefill chunk length (0 = automatic)")
+    ap.add_argument("--layout", choices=["head-major", "token-major"], default="head-major",
+                    help="prefill q/k/v/out layout: [B][H][N][D] or [B][N][H][D]")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the end-to-end leg")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="0 skips the CPU baseline")
@@ -213,10 +215,25 @@ def bench_prefill(args, dist, w, dev):
 
     q, k, v = I.device_prefill_inputs(w, dev)
     sl = torch.from_numpy(I.slopes_for(w)).to(dev)
-    out = torch.empty((w.B, w.H, w.N, w.E), dtype=torch.float32, device=dev)
+    token_major = args.layout == "token-major"
+    if token_major:
+        # [B][N][H][D] buffers, as a QKV projection writes them; the kernel
+        # reads them through strided views, with no transposing copy per step
+        q, k, v = (x.permute(0, 2, 1, 3).contiguous() for x in (q, k, v))
+        out = torch.empty((w.B, w.N, w.H, w.E), dtype=torch.float32, device=dev)
+    else:
+        out = torch.empty((w.B, w.H, w.N, w.E), dtype=torch.float32, device=dev)
+
+    def call(qx, kx, vx, ox):
+        if token_major:
+            tv = lambda x: x.permute(0, 2, 1, 3)
+            ops.fwd_strided(tv(qx), tv(kx), tv(vx), sl, tv(ox), chunk=args.chunk)
+        else:
+            ops.fwd(qx, kx, vx, sl, ox, chunk=args.chunk)
+
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
-        ops.fwd(q, k, v, sl, out, chunk=args.chunk)
+        call(q, k, v, out)
     torch.cuda.synchronize()
     assert ops.device_status(reset=True) == 0, "device-side wait timed out during warm-up"
     dist.barrier()
@@ -226,7 +243,7 @@ def bench_prefill(args, dist, w, dev):
     t_host0 = time.time()
     for i in range(args.steps):
         starts[i].record(stream)
-        ops.fwd(q, k, v, sl, out, chunk=args.chunk)
+        call(q, k, v, out)
         ends[i].record(stream)
     torch.cuda.synchronize()
     t_host1 = time.time()
@@ -252,7 +269,7 @@ def bench_prefill(args, dist, w, dev):
         dq.copy_(hq, non_blocking=True)
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
-        ops.fwd(dq, dk, dv, sl, out, chunk=args.chunk)
+        call(dq, dk, dv, out)
         hout.copy_(out, non_blocking=True)
 
     e2e_step()
@@ -379,6 +396,7 @@ def main_ours(args):
         "data": "synthetic (seeded torch generator on the device; q, k = SiLU(N(0,1)), v = N(0,1))",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "E": w.E,
                    "global_batch": w.B * dist.world, "seq_len": w.N, "chunk": args.chunk or "auto",
+                   "layout": args.layout,
                    "parallelism": f"replicas x{dist.world} (independent (b,h) problems, no collective)",
                    "l2": f"no flush: each step streams {bytes_launch / 1e9:.2f} GB, larger than the "
                          "126 MB L2"},

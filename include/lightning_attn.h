@@ -127,6 +127,29 @@ int lightning_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                int N, int D, int E, int chunk, void* stream);
 
 /*
+ * Prefill with caller-chosen strides, otherwise as lightning_attn_fwd_ex
+ * (same operation, decays, optional initial/final state and chunk length;
+ * bf16 q, k, v, fp32 out, D = E = 128).  For each of q, k, v and out,
+ * {stride_b, stride_h, stride_t} gives the element strides of its batch, head
+ * and token dimensions; the innermost dimension (d or e) is contiguous.  This
+ * takes the layouts a QKV projection produces without a transposing copy:
+ * token-major [B][N][H][D] (strides {N*H*D, D, H*D}) or views into one fused
+ * [B][N][3][H][D] buffer (strides {3*N*H*D, D, 3*H*D}, q, k, v H*D elements
+ * apart), and token-major outputs [B][N][H][E] (the layout of the layer's
+ * output projection input).  The pages show only the per-head computation;
+ * the layouts are this library's reading of how a model feeds it.
+ * Every stride times the element size (2 bytes for q, k, v; 4 for out) must be
+ * a non-negative multiple of 16 bytes below 2^40, and every pointer 16-byte
+ * aligned (else LA_ERR_ALIGN); NULL stride arrays give LA_ERR_NULL.  The
+ * elements of out must not overlap each other or the inputs (not checked).
+ */
+int lightning_attn_fwd_strided(const void* q, const void* k, const void* v, const float* slopes,
+                               const float* init_state, float* final_state, float* out, int B,
+                               int H, int N, int D, int E, const long long* q_strides,
+                               const long long* k_strides, const long long* v_strides,
+                               const long long* out_strides, int chunk, void* stream);
+
+/*
  * Prefill with fp32 inputs and output (same operation and layout as
  * lightning_attn_fwd, all tensors fp32).  D, E in {64, 128}.  CUDA-core fp32
  * arithmetic, for callers that need fp32-class accuracy.

@@ -262,9 +262,52 @@ __device__ __forceinline__ int next_work(const Params& p, int& n) {
   return blockIdx.x + gridDim.x * n++;
 }
 
+// Coordinates (beyond the column) of a tile of tokens [row, row + 128) of
+// head hh of batch bb in a 4-D tensor map whose outer dimensions are ordered
+// as `slots` says (see make_tmap_4d).
+struct TmaCoords {
+  int c1, c2, c3;
+};
+__device__ __forceinline__ TmaCoords tma_coords(int slots, int row, int hh, int bb) {
+  const int st = slots & 3, sh = (slots >> 2) & 3;
+  TmaCoords c;
+  c.c1 = st == 1 ? row : sh == 1 ? hh : bb;
+  c.c2 = st == 2 ? row : sh == 2 ? hh : bb;
+  c.c3 = st == 3 ? row : sh == 3 ? hh : bb;
+  return c;
+}
+
+// One 64-column half of a tile of 128 tokens of sequence seq (= bb * H + hh):
+// contiguous head-major tensors use 3-D maps [B*H][N][cols]; strided ones 4-D
+// maps (measured: the 4-D form costs a few percent, so it is only used when
+// the layout needs it).
+template <int RANK>
+__device__ __forceinline__ void tile_load(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                          int row, int seq, int hh, int bb, int slots,
+                                          uint64_t pol) {
+  if constexpr (RANK == 3) {
+    tma_load_3d(dst, map, bar, x, row, seq, pol);
+  } else {
+    const TmaCoords tc = tma_coords(slots, row, hh, bb);
+    tma_load_4d(dst, map, bar, x, tc.c1, tc.c2, tc.c3, pol);
+  }
+}
+
+template <int RANK>
+__device__ __forceinline__ void tile_store(const CUtensorMap* map, const void* src, int x, int row,
+                                           int seq, int hh, int bb, int slots, uint64_t pol) {
+  if constexpr (RANK == 3) {
+    tma_store_3d(map, src, x, row, seq, pol);
+  } else {
+    const TmaCoords tc = tma_coords(slots, row, hh, bb);
+    tma_store_4d(map, src, x, tc.c1, tc.c2, tc.c3, pol);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Producer: one thread issues every TMA load.
 // ---------------------------------------------------------------------------
+template <int RANK>
 __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
                          const CUtensorMap* tk, const CUtensorMap* tv) {
   const uint64_t pol_first = policy_evict_first();
@@ -272,14 +315,15 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
   uint32_t q_it = 0, k_it = 0, v_it = 0, w_it = 0;
   int n_items = 0;
   auto load = [&](int ring_f, int ring_e, uint32_t off, uint32_t& it, const CUtensorMap* tm,
-                  int row, int seq, uint64_t pol) -> bool {
+                  int tensor, int row, int seq, int hh, int bb, uint64_t pol) -> bool {
     const uint32_t s = it & 1u;
     if (it >= 2 && !wait_bar(c, p, ring_e + s, ((it >> 1) - 1) & 1u)) return false;
     uint8_t* dst = c.sm + off + s * TILE;
     LA_TRACE_EVENT(ring_f == B_QF ? 0 : ring_f == B_KF ? 1 : 2, it);
     mbar_arrive_expect_tx(&c.bar[ring_f + s], TILE);
-    tma_load_3d(dst, tm, &c.bar[ring_f + s], 0, row, seq, pol);
-    tma_load_3d(dst + PLANE, tm, &c.bar[ring_f + s], 64, row, seq, pol);
+    tile_load<RANK>(dst, tm, &c.bar[ring_f + s], 0, row, seq, hh, bb, p.cslot[tensor], pol);
+    tile_load<RANK>(dst + PLANE, tm, &c.bar[ring_f + s], 64, row, seq, hh, bb, p.cslot[tensor],
+                    pol);
     ++it;
     return true;
   };
@@ -320,6 +364,7 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
     ++w_it;
     Item it;
     if (!get_item(p, c.misc, w, it)) break;
+    const int hh = it.seq % p.H, bb = it.seq / p.H;
     bool ok = true;
     if (it.phase1) {
       for (int b = 0; b < it.nb && ok; ++b) {
@@ -331,10 +376,11 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
         uint8_t* dst = c.sm + p1_base(slot);
         uint64_t* full = &c.bar[B_P1F + slot];
         mbar_arrive_expect_tx(full, 2 * TILE);
-        tma_load_3d(dst, tk, full, 0, row, it.seq, pol_last);
-        tma_load_3d(dst + PLANE, tk, full, 64, row, it.seq, pol_last);
-        tma_load_3d(dst + TILE, tv, full, 0, row, it.seq, pol_last);
-        tma_load_3d(dst + TILE + PLANE, tv, full, 64, row, it.seq, pol_last);
+        tile_load<RANK>(dst, tk, full, 0, row, it.seq, hh, bb, p.cslot[1], pol_last);
+        tile_load<RANK>(dst + PLANE, tk, full, 64, row, it.seq, hh, bb, p.cslot[1], pol_last);
+        tile_load<RANK>(dst + TILE, tv, full, 0, row, it.seq, hh, bb, p.cslot[2], pol_last);
+        tile_load<RANK>(dst + TILE + PLANE, tv, full, 64, row, it.seq, hh, bb, p.cslot[2],
+                        pol_last);
         ++p1_it;
         pairs_pending = true;
       }
@@ -345,9 +391,9 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
     }
     for (int n = 0; n < (it.p2 ? it.nb : 0) && ok; ++n) {
       const int row = it.t0 + n * BLK;
-      ok = load(B_QF, B_QE, OFF_Q, q_it, tq, row, it.seq, pol_first) &&
-           load(B_KF, B_KE, OFF_K, k_it, tk, row, it.seq, pol_first) &&
-           load(B_VF, B_VE, OFF_V, v_it, tv, row, it.seq, pol_first);
+      ok = load(B_QF, B_QE, OFF_Q, q_it, tq, 0, row, it.seq, hh, bb, pol_first) &&
+           load(B_KF, B_KE, OFF_K, k_it, tk, 1, row, it.seq, hh, bb, pol_first) &&
+           load(B_VF, B_VE, OFF_V, v_it, tv, 2, row, it.seq, hh, bb, pol_first);
     }
     if (!ok) break;
   }
@@ -624,6 +670,7 @@ __device__ __forceinline__ void st_scan32(float* base, uint32_t r, uint32_t hf, 
                        __uint_as_float(x[4 * i + 2]), __uint_as_float(x[4 * i + 3])));
 }
 
+template <int RANK>
 __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
   const uint32_t t = threadIdx.x - 32u * Y_WARP0;  // 0..127
   const uint32_t r = t;                            // TMEM lane / tile row
@@ -820,8 +867,10 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
       fence_proxy_async_smem();
       if (!gsync(c, p, B_YSYNC, ys_n)) { ok = false; break; }
       if (leader) {
-        tma_store_3d(to, vtile_g, 0, row, it.seq, pol_out);
-        tma_store_3d(to, vtile_g + PLANE, 32, row, it.seq, pol_out);
+        tile_store<RANK>(to, vtile_g, 0, row, it.seq, it.seq % p.H, it.seq / p.H, p.cslot[3],
+                         pol_out);
+        tile_store<RANK>(to, vtile_g + PLANE, 32, row, it.seq, it.seq % p.H, it.seq / p.H,
+                         p.cslot[3], pol_out);
         bulk_commit_group();
         LA_TRACE_EVENT(23, g);
       }
@@ -839,8 +888,10 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
       fence_proxy_async_smem();
       if (!gsync(c, p, B_YSYNC, ys_n)) { ok = false; break; }
       if (leader) {
-        tma_store_3d(to, vtile_g, 64, row, it.seq, pol_out);
-        tma_store_3d(to, vtile_g + PLANE, 96, row, it.seq, pol_out);
+        tile_store<RANK>(to, vtile_g, 64, row, it.seq, it.seq % p.H, it.seq / p.H, p.cslot[3],
+                         pol_out);
+        tile_store<RANK>(to, vtile_g + PLANE, 96, row, it.seq, it.seq % p.H, it.seq / p.H,
+                         p.cslot[3], pol_out);
         bulk_commit_group();
         LA_TRACE_EVENT(26, g);
         bulk_wait_group_read<0>();
@@ -857,6 +908,8 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
 
 // 14 warps on 4 SM sub-partitions (16K registers each, at most 4 warps on one)
 // leave up to 128 registers per thread.
+// RANK: 3 for contiguous head-major q, k, v, out; 4 for strided layouts.
+template <int RANK>
 __global__ void __launch_bounds__(THREADS, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
@@ -921,14 +974,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   c.tmem = c.misc[0];
 
   if (warp == PRODUCER_WARP) {
-    if (lane_id() == 0) producer(c, p, &tq, &tk, &tv);
+    if (lane_id() == 0) producer<RANK>(c, p, &tq, &tk, &tv);
   } else if (warp == MMA_WARP) {
     if (lane_id() == 0) mma_issuer(c, p);
     __syncwarp();
   } else if (warp < Y_WARP0) {
     group_x(c, p);
   } else {
-    group_y(c, p, &to);
+    group_y<RANK>(c, p, &to);
   }
 
   tc_fence_before();

@@ -31,6 +31,7 @@ struct Params {
   int F, G2;                  // split scan: blocks of each sequence in the local-state pass;
                               // CTAs whose outputs cover that part
   long long P;                // split scan: nseq * F
+  int cslot[4];               // q, k, v, out tensor maps: where t, h, b sit (make_tmap_4d)
   unsigned long long wait_limit_ns;
 };
 

@@ -177,10 +177,88 @@ void set_scratch(const Plan& pl, void* scratch, la::fwd::Params& p) {
   p.prefix = reinterpret_cast<float*>(static_cast<char*>(scratch) + pl.ctrl);
 }
 
+// Element strides {b, h, t} of q, k, v and out (d or e contiguous).
+struct Strides {
+  long long s[4][3];
+};
+
+Strides contiguous_strides(int H, int N, int D, int E) {
+  Strides st;
+  const long long w[4] = {D, D, E, E};
+  for (int i = 0; i < 4; ++i) {
+    st.s[i][2] = w[i];
+    st.s[i][1] = static_cast<long long>(N) * w[i];
+    st.s[i][0] = static_cast<long long>(H) * N * w[i];
+  }
+  return st;
+}
+
+// TMA needs every stride in bytes to be a multiple of 16 and below 2^40.
+bool strides_ok(const Strides& st) {
+  const int eb[4] = {2, 2, 2, 4};
+  for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < 3; ++j) {
+      const long long b = st.s[i][j] * eb[i];
+      if (st.s[i][j] < 0 || b % 16 != 0 || b >= (1ll << 40)) return false;
+    }
+  return true;
+}
+
+// The four tensor maps of the bf16 prefill: 3-D [B*H][N][cols] maps when
+// every tensor is contiguous head-major, else 4-D maps (p.cslot says where t,
+// h and b went).  *rank receives 3 or 4.
+bool build_maps(const void* q, const void* k, const void* v, const float* out, int B, int H, int N,
+                const Strides& st, CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv,
+                CUtensorMap* to, la::fwd::Params& p, int* rank) {
+  const Strides cont = contiguous_strides(H, N, 128, 128);
+  bool contiguous = true;
+  for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < 3; ++j) {
+      const bool unused = (j == 0 && B == 1) || (j == 1 && H == 1);  // extent-1 dimension
+      contiguous = contiguous && (unused || st.s[i][j] == cont.s[i][j]);
+    }
+  if (contiguous) {
+    *rank = 3;
+    const uint64_t nseq = static_cast<uint64_t>(B) * H;
+    return la::make_tmap_3d(tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) &&
+           la::make_tmap_3d(tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) &&
+           la::make_tmap_3d(tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) &&
+           la::make_tmap_3d(to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, N, nseq, 32, 128);
+  }
+  *rank = 4;
+  const uint64_t ext[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(H),
+                           static_cast<uint64_t>(B)};
+  CUtensorMap* maps[4] = {tq, tk, tv, to};
+  const void* bases[4] = {q, k, v, out};
+  for (int i = 0; i < 4; ++i) {
+    const uint64_t str[3] = {static_cast<uint64_t>(st.s[i][2]), static_cast<uint64_t>(st.s[i][1]),
+                             static_cast<uint64_t>(st.s[i][0])};
+    const bool f32 = i == 3;
+    if (!la::make_tmap_4d(maps[i], bases[i],
+                          f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                          f32 ? 4 : 2, 128, ext, str, f32 ? 32 : 64, 128, &p.cslot[i]))
+      return false;
+  }
+  return true;
+}
+
+// Launches the prefill kernel for the map rank (sets the shared-memory
+// attribute on every call: it belongs to the current device's context).
+int launch_fwd(int rank, int grid, cudaStream_t stream, const CUtensorMap& tq,
+               const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+               const la::fwd::Params& p) {
+  auto kern = rank == 3 ? la::fwd::fwd_bf16_kernel<3> : la::fwd::fwd_bf16_kernel<4>;
+  const cudaError_t attr =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::fwd::SMEM_BYTES);
+  if (attr != cudaSuccess) return cuda_fail(attr);
+  kern<<<grid, la::fwd::THREADS, la::fwd::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+  return launch_status();
+}
+
 int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slopes,
                   const float* init_state, float* final_state, float* out, int B, int H, int N,
-                  int D, int E, int chunk, void* stream_ptr, int first_chunk = 0,
-                  unsigned long long wait_limit_ns = kWaitLimitNs) {
+                  int D, int E, int chunk, void* stream_ptr, const Strides* strides = nullptr,
+                  int first_chunk = 0, unsigned long long wait_limit_ns = kWaitLimitNs) {
   if (!q || !k || !v || !slopes || !out) return LA_ERR_NULL;
   if (!dims_ok(B, H, N, D, E)) return LA_ERR_SHAPE;
   if (D != 128 || E != 128) return LA_ERR_UNSUPPORTED;
@@ -194,14 +272,13 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   const Plan pl = make_plan(nseq, N, sms, chunk);
   if (pl.total >= (1ll << 31)) return LA_ERR_SHAPE;
 
-  CUtensorMap tq, tk, tv, to;
-  if (!la::make_tmap_3d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
-      !la::make_tmap_3d(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
-      !la::make_tmap_3d(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
-      !la::make_tmap_3d(&to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, N, nseq, 32, 128))
-    return LA_ERR_CUDA;
-
+  const Strides st = strides ? *strides : contiguous_strides(H, N, D, E);
+  if (!strides_ok(st)) return LA_ERR_ALIGN;
   la::fwd::Params p{};
+  CUtensorMap tq, tk, tv, to;
+  int rank = 3;
+  if (!build_maps(q, k, v, out, B, H, N, st, &tq, &tk, &tv, &to, p, &rank)) return LA_ERR_CUDA;
+
   p.slopes = slopes;
   p.init_state = init_state;
   p.final_state = final_state;
@@ -225,18 +302,7 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
     set_scratch(pl, scratch, p);
   }
 
-  // set on every call: the attribute belongs to the current device's context
-  const cudaError_t attr =
-      cudaFuncSetAttribute(la::fwd::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           la::fwd::SMEM_BYTES);
-  int rc = LA_OK;
-  if (attr != cudaSuccess) {
-    rc = cuda_fail(attr);
-  } else {
-    la::fwd::fwd_bf16_kernel<<<pl.grid, la::fwd::THREADS, la::fwd::SMEM_BYTES, stream>>>(
-        tq, tk, tv, to, p);
-    rc = launch_status();
-  }
+  int rc = launch_fwd(rank, pl.grid, stream, tq, tk, tv, to, p);
   if (scratch) {
     const cudaError_t e = cudaFreeAsync(scratch, stream);
     if (e != cudaSuccess && rc == LA_OK) rc = cuda_fail(e);
@@ -296,14 +362,13 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
   if (pl.total >= (1ll << 31)) return LA_ERR_SHAPE;
   if (pl.bytes > LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_WORKSPACE;
 
+  la::fwd::Params p{};
   CUtensorMap tq, tk, tv, to;
-  if (!la::make_tmap_3d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
-      !la::make_tmap_3d(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
-      !la::make_tmap_3d(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) ||
-      !la::make_tmap_3d(&to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, N, nseq, 32, 128))
+  int rank = 3;
+  if (!build_maps(q, k, v, out, B, H, N, contiguous_strides(H, N, D, E), &tq, &tk, &tv, &to, p,
+                  &rank))
     return LA_ERR_CUDA;
 
-  la::fwd::Params p{};
   p.slopes = slopes;
   p.status = status_word();
   if (!p.status) return LA_ERR_CUDA;
@@ -321,13 +386,7 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
     if (e != cudaSuccess) return cuda_fail(e);
     set_scratch(pl, scratch, p);
   }
-  const cudaError_t attr =
-      cudaFuncSetAttribute(la::fwd::fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           la::fwd::SMEM_BYTES);
-  if (attr != cudaSuccess) return cuda_fail(attr);
-  la::fwd::fwd_bf16_kernel<<<pl.grid, la::fwd::THREADS, la::fwd::SMEM_BYTES, stream>>>(tq, tk, tv,
-                                                                                     to, p);
-  return launch_status();
+  return launch_fwd(rank, pl.grid, stream, tq, tk, tv, to, p);
 }
 
 template <int D, int E>
@@ -367,13 +426,27 @@ int lightning_attn_fwd_ex(const void* q, const void* k, const void* v, const flo
                        stream);
 }
 
+int lightning_attn_fwd_strided(const void* q, const void* k, const void* v, const float* slopes,
+                               const float* init_state, float* final_state, float* out, int B,
+                               int H, int N, int D, int E, const long long* q_strides,
+                               const long long* k_strides, const long long* v_strides,
+                               const long long* out_strides, int chunk, void* stream) {
+  if (!q_strides || !k_strides || !v_strides || !out_strides) return LA_ERR_NULL;
+  Strides st;
+  const long long* src[4] = {q_strides, k_strides, v_strides, out_strides};
+  for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < 3; ++j) st.s[i][j] = src[i][j];
+  return fwd_bf16_impl(q, k, v, slopes, init_state, final_state, out, B, H, N, D, E, chunk,
+                       stream, &st);
+}
+
 int lightning_attn_fault_test_scan_stall(const void* q, const void* k, const void* v,
                                          const float* slopes, float* out, int B, int H, int N,
                                          int chunk, unsigned int wait_limit_ms, void* stream) {
   if (chunk <= 0 || N <= chunk) return LA_ERR_SHAPE;  // needs at least two chunks
   if (wait_limit_ms == 0 || wait_limit_ms > 10000) return LA_ERR_SHAPE;
   return fwd_bf16_impl(q, k, v, slopes, nullptr, nullptr, out, B, H, N, 128, 128, chunk, stream,
-                       /*first_chunk=*/1, 1000000ull * wait_limit_ms);
+                       /*strides=*/nullptr, /*first_chunk=*/1, 1000000ull * wait_limit_ms);
 }
 
 int lightning_attn_fwd_noalloc(const void* q, const void* k, const void* v, const float* slopes,

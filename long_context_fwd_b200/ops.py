@@ -36,6 +36,8 @@ SIGNATURES = {
     "lightning_attn_last_cuda_error": [],
     "lightning_attn_device_status": [_P, _I],
     "lightning_attn_fwd_plan": [_I, _I, _I, _I, _I, _P, _P, _I, _P],
+    "lightning_attn_fwd_strided": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P,
+                                   _I, _P],
 }
 
 
@@ -127,6 +129,46 @@ def fwd(q, k, v, slopes, out=None, *, init_state=None, final_state=None, chunk: 
             None if final_state is None else final_state.data_ptr(),
             out.data_ptr(), B, H, N, D, E, int(chunk), _stream_handle(stream))
         _check("lightning_attn_fwd_ex", rc)
+    return out
+
+
+def _need_view(t: torch.Tensor, name: str, dtype, shape):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.stride(-1) != 1:
+        raise ValueError(f"{name}: the last dimension must be contiguous")
+
+
+def fwd_strided(q, k, v, slopes, out, *, init_state=None, final_state=None, chunk: int = 0,
+                stream=None) -> torch.Tensor:
+    """Prefill on strided views: q, k [B,H,N,D] and v [B,H,N,E] bf16, out [B,H,N,E] fp32,
+    each with any (b, h, t) strides and a contiguous last dimension -- e.g.
+    ``qt.permute(0, 2, 1, 3)`` of a token-major ``qt`` [B,N,H,D], or slices of a
+    fused [B,N,3,H,D] projection output."""
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    _need_view(q, "q", torch.bfloat16, (B, H, N, D))
+    _need_view(k, "k", torch.bfloat16, (B, H, N, D))
+    _need_view(v, "v", torch.bfloat16, (B, H, N, E))
+    _need_view(out, "out", torch.float32, (B, H, N, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    for name, st in (("init_state", init_state), ("final_state", final_state)):
+        if st is not None:
+            _need(st, name, torch.float32, (B, H, D, E))
+    arr = [(ctypes.c_longlong * 3)(*t.stride()[:3]) for t in (q, k, v, out)]
+    rc = lib().lightning_attn_fwd_strided(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), slopes.data_ptr(),
+        None if init_state is None else init_state.data_ptr(),
+        None if final_state is None else final_state.data_ptr(),
+        out.data_ptr(), B, H, N, D, E, *[ctypes.cast(a, ctypes.c_void_p) for a in arr],
+        int(chunk), _stream_handle(stream))
+    _check("lightning_attn_fwd_strided", rc)
     return out
 
 

@@ -109,3 +109,21 @@ def test_noalloc_rejects_oversized_scratch_on_host(lib):
     # before any launch.
     f = lib.lightning_attn_fwd_noalloc
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 200, 1024, 128, 128, 128, None) == 7
+
+
+def test_strided_validation(lib):
+    f = lib.lightning_attn_fwd_strided
+    C = ctypes.c_longlong * 3
+    ok = C(4 * 64 * 128, 64 * 128, 128)  # token-major-like, all multiples of 16 bytes
+    ok_o = C(4 * 64 * 128, 64 * 128, 128)
+    args = lambda qs, ks, vs, os: (FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 4, 64, 128, 128,
+                                   qs, ks, vs, os, 0, None)
+    assert f(*args(None, ok, ok, ok_o)) == LA_ERR_NULL
+    bad_t = C(4 * 64 * 128, 64 * 128, 100)  # 200-byte token stride
+    assert f(*args(bad_t, ok, ok, ok_o)) == LA_ERR_ALIGN
+    neg = C(4 * 64 * 128, -128, 128)
+    assert f(*args(ok, neg, ok, ok_o)) == LA_ERR_ALIGN
+    bad_o = C(4 * 64 * 128, 64 * 128, 130)  # 520-byte fp32 token stride
+    assert f(*args(ok, ok, ok, bad_o)) == LA_ERR_ALIGN
+    assert f(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 4, 64, 64, 128, ok, ok, ok, ok_o, 0,
+             None) == LA_ERR_UNSUPPORTED
