@@ -62,13 +62,17 @@ typedef enum {
  * Prefill, bf16 inputs, fp32 output.
  *   q, k : bf16 [B][H][N][D]      v : bf16 [B][H][N][E]
  *   slopes: fp32 [H], lambda_h    out: fp32 [B][H][N][E] (fully overwritten)
- * Zero initial state.  D = E = 128 is the supported head geometry (the
- * "128x128 state per head" of the MiniMax-M1 entry, linear-layer field);
- * other D, E return LA_ERR_UNSUPPORTED.  Any N >= 1.
+ * Zero initial state.  D, E in {64, 128} (the model's geometry is the
+ * "128x128 state per head" of the MiniMax-M1 entry, linear-layer field; a
+ * 64-wide q/k or v runs on the same 128-wide tiles with the missing columns
+ * zero-filled by the tensor maps, which is exact); other D, E return
+ * LA_ERR_UNSUPPORTED.  Any N >= 1.
  * Runs on tcgen05 tensor cores (bf16 operands, fp32 accumulation, fp32 state
- * carried on chip).  Long sequences are split into chunks processed in parallel
- * with a chained state scan; the scan scratch (about 128 KiB per (b, h)) is
- * taken with cudaMallocAsync / cudaFreeAsync on `stream`.
+ * carried on chip).  Work is spread over all SMs: long sequences are split
+ * into parts whose entering states come from a state scan or a hand-over;
+ * the scratch (at most 2 states of 64 KiB per SM, or per (b, h) with an
+ * explicit chunk length) is taken with cudaMallocAsync / cudaFreeAsync on
+ * `stream`.
  */
 int lightning_attn_fwd(const void* q, const void* k, const void* v,
                        const float* slopes, float* out,
@@ -129,7 +133,7 @@ int lightning_attn_fwd_noalloc(const void* q, const void* k, const void* v,
 /*
  * Prefill with caller-chosen strides, otherwise as lightning_attn_fwd_ex
  * (same operation, decays, optional initial/final state and chunk length;
- * bf16 q, k, v, fp32 out, D = E = 128).  For each of q, k, v and out,
+ * bf16 q, k, v, fp32 out, D, E in {64, 128}).  For each of q, k, v and out,
  * {stride_b, stride_h, stride_t} gives the element strides of its batch, head
  * and token dimensions; the innermost dimension (d or e) is contiguous.  This
  * takes the layouts a QKV projection produces without a transposing copy:

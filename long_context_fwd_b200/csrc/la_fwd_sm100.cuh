@@ -677,7 +677,11 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
   const uint32_t lane_base = ((t >> 5) * 32u) << 16;
   const uint32_t t_kv = c.tmem + lane_base + TM_KV;
   const uint32_t t_o = c.tmem + lane_base + TM_O;
-  const int64_t row_off = static_cast<int64_t>(r) * HD;
+  // the caller's states are [seq][D][E]; rows r >= D of the 128 x 128 TMEM
+  // state are zero (zero-filled K columns) and never read or written
+  const int64_t row_off = static_cast<int64_t>(r) * p.E;
+  const bool row_in = static_cast<int>(r) < p.D;
+  const int64_t state_elems = static_cast<int64_t>(p.D) * p.E;
   const bool leader = (t == 0);
   const uint64_t pol_out = policy_evict_first();
   uint32_t v_it = 0, w_it = 0, gb = 0, agg_n = 0, ys_n = 0;
@@ -731,8 +735,8 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     }
     // the caller's initial state enters at block 0 of a sequence (or through
     // the chain); never into a local state
-    if (p.init_state && it.p2 && (!it.enter || chain))
-      init_src = p.init_state + static_cast<int64_t>(it.seq) * (HD * HD) + row_off;
+    if (p.init_state && it.p2 && (!it.enter || chain) && row_in)
+      init_src = p.init_state + static_cast<int64_t>(it.seq) * state_elems + row_off;
     if (leader) LA_TRACE_EVENT(16, w_it);
     if (it.phase1 && !cwait(c, p, B_AGG_FULL, agg_n++ & 1u)) break;
     if (leader) LA_TRACE_EVENT(17, w_it);
@@ -746,7 +750,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         uint32_t prev[32];
         if (scan_src) {
           ld_scan32(scan_src, r, q >> 1, q & 1u, prev);
-        } else if (init_src) {
+        } else if (init_src && 32 * static_cast<int>(q) < p.E) {
           ld_global32(init_src + 32 * q, prev);
         } else {
 #pragma unroll
@@ -800,9 +804,9 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
 
     // where the state after the item's last block goes: the caller's final
     // state (row layout) or a balanced split's hand-over slot (scan layout)
-    float* const fin_dst =
-        it.last && p.final_state ? p.final_state + static_cast<int64_t>(it.seq) * (HD * HD) + row_off
-                                 : nullptr;
+    float* const fin_dst = it.last && p.final_state && row_in
+                               ? p.final_state + static_cast<int64_t>(it.seq) * state_elems + row_off
+                               : nullptr;
     float* const pub_dst = it.publish ? p.prefix + static_cast<int64_t>(it.pub_slot) * (HD * HD) : nullptr;
     int* const pub_flag = it.publish ? p.flags + it.pub_slot : nullptr;
     const int pub_val = it.pub_val;
@@ -829,7 +833,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
             store_half_bf16(kvb_row(q), r, q & 1u, kv, 1.f);
             tmem_st32_scaled(t_kv + 32u * q, kv, gnext);
           } else if (fin) {
-            st_global32(fin_dst + 32 * q, kv);
+            if (32 * static_cast<int>(q) < p.E) st_global32(fin_dst + 32 * q, kv);
           } else if (pub) {
             st_scan32(pub_dst, r, q >> 1, q & 1u, kv);
           }

@@ -32,6 +32,8 @@ struct Params {
                               // CTAs whose outputs cover that part
   long long P;                // split scan: nseq * F
   int cslot[4];               // q, k, v, out tensor maps: where t, h, b sit (make_tmap_4d)
+  int D, E;                   // the caller's head dimensions (64 or 128; tiles are 128 wide,
+                              // the tensor maps zero-fill the columns past D or E)
   unsigned long long wait_limit_ns;
 };
 

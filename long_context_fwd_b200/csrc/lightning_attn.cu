@@ -208,9 +208,15 @@ bool strides_ok(const Strides& st) {
 // every tensor is contiguous head-major, else 4-D maps (p.cslot says where t,
 // h and b went).  *rank receives 3 or 4.
 bool build_maps(const void* q, const void* k, const void* v, const float* out, int B, int H, int N,
-                const Strides& st, CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv,
+                int D, int E, const Strides& st, CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv,
                 CUtensorMap* to, la::fwd::Params& p, int* rank) {
-  const Strides cont = contiguous_strides(H, N, 128, 128);
+  // Column extents D and E: a 64-wide tensor leaves the second 64-column half
+  // of every 128-wide tile outside the map, so TMA fills it with zeros (no
+  // memory traffic) and clips stores there; zero columns add nothing to any
+  // product, so the 128 x 128 kernel computes the D x E result exactly.
+  p.D = D;
+  p.E = E;
+  const Strides cont = contiguous_strides(H, N, D, E);
   bool contiguous = true;
   for (int i = 0; i < 4; ++i)
     for (int j = 0; j < 3; ++j) {
@@ -220,10 +226,10 @@ bool build_maps(const void* q, const void* k, const void* v, const float* out, i
   if (contiguous) {
     *rank = 3;
     const uint64_t nseq = static_cast<uint64_t>(B) * H;
-    return la::make_tmap_3d(tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) &&
-           la::make_tmap_3d(tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) &&
-           la::make_tmap_3d(tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, N, nseq, 64, 128) &&
-           la::make_tmap_3d(to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 128, N, nseq, 32, 128);
+    return la::make_tmap_3d(tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, nseq, 64, 128) &&
+           la::make_tmap_3d(tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, nseq, 64, 128) &&
+           la::make_tmap_3d(tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, nseq, 64, 128) &&
+           la::make_tmap_3d(to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, E, N, nseq, 32, 128);
   }
   *rank = 4;
   const uint64_t ext[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(H),
@@ -236,7 +242,7 @@ bool build_maps(const void* q, const void* k, const void* v, const float* out, i
     const bool f32 = i == 3;
     if (!la::make_tmap_4d(maps[i], bases[i],
                           f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                          f32 ? 4 : 2, 128, ext, str, f32 ? 32 : 64, 128, &p.cslot[i]))
+                          f32 ? 4 : 2, i < 2 ? D : E, ext, str, f32 ? 32 : 64, 128, &p.cslot[i]))
       return false;
   }
   return true;
@@ -261,7 +267,7 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
                   int first_chunk = 0, unsigned long long wait_limit_ns = kWaitLimitNs) {
   if (!q || !k || !v || !slopes || !out) return LA_ERR_NULL;
   if (!dims_ok(B, H, N, D, E)) return LA_ERR_SHAPE;
-  if (D != 128 || E != 128) return LA_ERR_UNSUPPORTED;
+  if ((D != 64 && D != 128) || (E != 64 && E != 128)) return LA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(slopes) ||
       (init_state && !aligned16(init_state)) || (final_state && !aligned16(final_state)))
     return LA_ERR_ALIGN;
@@ -277,7 +283,8 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   la::fwd::Params p{};
   CUtensorMap tq, tk, tv, to;
   int rank = 3;
-  if (!build_maps(q, k, v, out, B, H, N, st, &tq, &tk, &tv, &to, p, &rank)) return LA_ERR_CUDA;
+  if (!build_maps(q, k, v, out, B, H, N, D, E, st, &tq, &tk, &tv, &to, p, &rank))
+    return LA_ERR_CUDA;
 
   p.slopes = slopes;
   p.init_state = init_state;
@@ -343,7 +350,7 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
                           void* stream_ptr) {
   if (!q || !k || !v || !slopes || !out) return LA_ERR_NULL;
   if (!dims_ok(B, H, N, D, E)) return LA_ERR_SHAPE;
-  if (D != 128 || E != 128) return LA_ERR_UNSUPPORTED;
+  if ((D != 64 && D != 128) || (E != 64 && E != 128)) return LA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(slopes))
     return LA_ERR_ALIGN;
   if (chunk < 0 || (chunk % 128) != 0) return LA_ERR_SHAPE;
@@ -365,8 +372,8 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
   la::fwd::Params p{};
   CUtensorMap tq, tk, tv, to;
   int rank = 3;
-  if (!build_maps(q, k, v, out, B, H, N, contiguous_strides(H, N, D, E), &tq, &tk, &tv, &to, p,
-                  &rank))
+  if (!build_maps(q, k, v, out, B, H, N, D, E, contiguous_strides(H, N, D, E), &tq, &tk, &tv, &to,
+                  p, &rank))
     return LA_ERR_CUDA;
 
   p.slopes = slopes;

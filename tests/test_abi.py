@@ -56,7 +56,7 @@ def test_fwd_validation(lib):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 128, 128, None) == LA_ERR_SHAPE
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 128, 128, None) == LA_ERR_SHAPE
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, -3, 8, 128, 128, None) == LA_ERR_SHAPE
-    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 128, None) == LA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 96, 128, None) == LA_ERR_UNSUPPORTED
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 128, 96, None) == LA_ERR_UNSUPPORTED
     assert f(FAKE + 8, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_ALIGN
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE + 4, 1, 1, 8, 128, 128, None) == LA_ERR_ALIGN
@@ -125,5 +125,5 @@ def test_strided_validation(lib):
     assert f(*args(ok, neg, ok, ok_o)) == LA_ERR_ALIGN
     bad_o = C(4 * 64 * 128, 64 * 128, 130)  # 520-byte fp32 token stride
     assert f(*args(ok, ok, ok, bad_o)) == LA_ERR_ALIGN
-    assert f(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 4, 64, 64, 128, ok, ok, ok, ok_o, 0,
+    assert f(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 4, 64, 32, 128, ok, ok, ok, ok_o, 0,
              None) == LA_ERR_UNSUPPORTED

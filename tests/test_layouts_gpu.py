@@ -21,8 +21,8 @@ pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
 
 
-def _case(B, H, N, seed):
-    w = I.Workload(f"layout{seed}", B, H, N, 128, 128, "bf16", index=500 + seed)
+def _case(B, H, N, seed, D=128, E=128):
+    w = I.Workload(f"layout{seed}", B, H, N, D, E, "bf16", index=500 + seed)
     q, k, v = I.prefill_inputs(w)
     sl = I.alibi_slopes(H)
     sl[::3] = 0.0
@@ -109,3 +109,17 @@ def test_token_major_initial_and_final_state():
     ref, sref = oracle.recurrent(q, k, v, sl, s0=s0.astype(np.float64), return_state=True)
     assert rel(out_tm.permute(0, 2, 1, 3).cpu().numpy(), ref) <= TOL_BF16
     assert rel(fin.cpu().numpy(), sref) <= TOL_BF16
+
+
+def test_token_major_with_64_wide_q_k():
+    B, H, N, D, E = 1, 64, 2000, 64, 128
+    q, k, v, sl = _case(B, H, N, seed=13, D=D, E=E)
+    _, qv = _token_major(q)
+    _, kv = _token_major(k)
+    _, vv = _token_major(v)
+    out_tm = torch.empty((B, N, H, E), dtype=torch.float32, device=DEV)
+    ops.fwd_strided(qv, kv, vv, f32_to_dev(sl, DEV), out_tm.permute(0, 2, 1, 3))
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0
+    ref = oracle.recurrent(q, k, v, sl)
+    assert rel(out_tm.permute(0, 2, 1, 3).cpu().numpy(), ref) <= TOL_BF16

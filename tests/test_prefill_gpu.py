@@ -186,6 +186,50 @@ def test_bf16_split_scan_initial_and_final_state():
     assert worst_head(fin.cpu().numpy(), sref) <= TOL_BF16
 
 
+# D != E on the tensor-core path: 64-wide q/k or v run on the 128-wide tiles
+# with the missing columns zero-filled by the tensor maps.  Whole sequences,
+# explicit chunks, the split scan and the hand-over; ragged ends.
+GEOMETRY_CASES = [
+    # B, H, N, D, E, chunk
+    (1, 3, 1000, 64, 128, 0),
+    (2, 2, 777, 128, 64, 0),
+    (1, 4, 3000, 64, 64, 512),
+    (1, 64, 2500, 64, 128, 0),
+    (2, 80, 1100, 128, 64, 0),
+]
+
+
+def _geo_case(B, H, N, D, E, seed):
+    w = I.Workload(f"geo{seed}", B, H, N, D, E, "bf16", index=600 + seed)
+    q, k, v = I.prefill_inputs(w)
+    sl = I.alibi_slopes(H)
+    sl[1::4] = 0.0
+    return q, k, v, sl
+
+
+@pytest.mark.parametrize("B,H,N,D,E,chunk", GEOMETRY_CASES)
+def test_bf16_head_geometries(B, H, N, D, E, chunk):
+    q, k, v, sl = _geo_case(B, H, N, D, E, seed=D + E + H)
+    assert q.shape[-1] == D and v.shape[-1] == E
+    got = _run(q, k, v, sl, chunk=chunk)
+    assert got.shape == (B, H, N, E)
+    ref = oracle.recurrent(q, k, v, sl)
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("B,H,N,D,E", [(1, 3, 1500, 64, 128), (1, 64, 1200, 128, 64),
+                                       (1, 2, 900, 64, 64)])
+def test_bf16_head_geometries_initial_and_final_state(B, H, N, D, E):
+    q, k, v, sl = _geo_case(B, H, N, D, E, seed=D + 2 * E + H)
+    s0 = (np.random.default_rng(3).standard_normal((B, H, D, E)) * 0.02).astype(np.float32)
+    fin = torch.zeros((B, H, D, E), dtype=torch.float32, device=DEV)
+    got = _run(q, k, v, sl, init_state=f32_to_dev(s0, DEV), final_state=fin)
+    ref, sref = oracle.recurrent(q, k, v, sl, s0=s0.astype(np.float64), return_state=True)
+    assert rel(got, ref) <= TOL_BF16
+    assert rel(fin.cpu().numpy(), sref) <= TOL_BF16
+
+
 def test_bf16_prefill_then_decode_continues_sequence():
     B, H, N, T = 2, 2, 700, 6
     w = I.Workload("handoff", B, H, N + T, 128, 128, "bf16", index=140)
