@@ -89,6 +89,24 @@ def alibi_slopes(H: int) -> np.ndarray:
     return np.power(2.0, -8.0 * (h + 1.0) / H).astype(np.float32)
 
 
+def depth_scaled_slopes(H: int, layer: int, n_layers: int) -> np.ndarray:
+    """Per-head decay rates of the layer at depth `layer` (0-based) of a model
+    with `n_layers` layers: the ALiBi-style rates scaled down linearly with
+    depth, lambda_h * (1 - layer / (n_layers - 1)), as float32.
+
+    "MiniMax-M1" model entry, linear-layer field: per-head exponential decay
+    with ALiBi-style slopes scaled down linearly with depth.  The field gives no
+    formula; this reading runs the factor from 1 at the first layer to 0 at the
+    last (whose Lightning layer, if it is one, is then plain causal linear
+    attention), counting every layer of the model.
+    """
+    if not 0 <= layer < n_layers:
+        raise ValueError(f"layer {layer} outside [0, {n_layers})")
+    factor = 1.0 if n_layers == 1 else 1.0 - layer / (n_layers - 1)
+    h = np.arange(H, dtype=np.float64)
+    return (np.power(2.0, -8.0 * (h + 1.0) / H) * factor).astype(np.float32)
+
+
 def slopes_for(w: Workload) -> np.ndarray:
     """The workload's per-head slopes (float32 [H])."""
     s = alibi_slopes(w.H)

@@ -14,6 +14,19 @@ def test_alibi_slopes_values():
     np.testing.assert_allclose(I.alibi_slopes(2), [2.0 ** -4, 2.0 ** -8], rtol=1e-7)
 
 
+def test_depth_scaled_slopes():
+    H, L = 64, 80
+    np.testing.assert_array_equal(I.depth_scaled_slopes(H, 0, L), I.alibi_slopes(H))
+    assert np.all(I.depth_scaled_slopes(H, L - 1, L) == 0.0)
+    per = np.stack([I.depth_scaled_slopes(H, l, L).astype(np.float64) for l in range(L)])
+    # linear in depth: constant first difference, every head
+    d = np.diff(per, axis=0)
+    np.testing.assert_allclose(d, np.broadcast_to(d[0], d.shape), rtol=1e-5, atol=1e-9)
+    assert np.all(d <= 0)
+    np.testing.assert_allclose(per[40], per[0] * (1 - 40 / 79), rtol=1e-6)
+    np.testing.assert_array_equal(I.depth_scaled_slopes(8, 0, 1), I.alibi_slopes(8))
+
+
 def test_zero_decay_heads():
     s = I.slopes_for(I.PREFILL_32K)
     zero = np.flatnonzero(s == 0.0)

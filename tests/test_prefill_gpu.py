@@ -230,6 +230,18 @@ def test_bf16_head_geometries_initial_and_final_state(B, H, N, D, E):
     assert rel(fin.cpu().numpy(), sref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("layer", [0, 41, 79])
+def test_bf16_depth_scaled_slopes(layer):
+    """Slopes of layer `layer` of an 80-layer model (the last one decays nothing)."""
+    B, H, N = 1, 16, 1500
+    sl = I.depth_scaled_slopes(H, layer, 80)
+    q, k, v, _ = _bf16_case(B, H, N, [0.0] * H, seed=70 + layer)
+    got = _run(q, k, v, sl)
+    ref = oracle.recurrent(q, k, v, sl)
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+
+
 def test_bf16_prefill_then_decode_continues_sequence():
     B, H, N, T = 2, 2, 700, 6
     w = I.Workload("handoff", B, H, N + T, 128, 128, "bf16", index=140)
