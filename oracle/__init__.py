@@ -18,7 +18,9 @@ What is computed (one problem per (b, h), layout [B][H][N][*]):
 after the "MiniMax-M1" model entry (archdb), linear/SSM layer configuration
 field (per-head exponential decay with ALiBi-style slopes, 128x128 state per
 head), and "MiniMax-01" (redeep.blog), "What Makes 1M Context Hard"
-(linear-complexity attention variant).
+(linear-complexity attention variant).  For training with long contexts (the
+abstract: 1M tokens in training) it also gives the anti-causal sum and the
+gradients of L = sum_t dout_t . o_t with respect to q, k and v.
 """
 from __future__ import annotations
 
@@ -63,8 +65,18 @@ def _load():
             lib.la_oracle_blocked.argtypes = [P, P, P, I, P, I64, P, I64, I64, I64, I64, I64, I]
             lib.la_oracle_decode_step.argtypes = [P, P, P, I, P, P, P, I64, I64, I64, I64, I]
             lib.la_oracle_max_threads.argtypes = []
+            lib.la_oracle_masked_anticausal.argtypes = [P, P, P, I, P, P, I64, I64, I64, I64, I64,
+                                                        I]
+            lib.la_oracle_recurrent_anticausal.argtypes = [P, P, P, I, P, P, P, P, I64, I64, I64,
+                                                           I64, I64, I]
+            lib.la_oracle_backward_masked.argtypes = [P, P, P, P, I, P, P, P, P, I64, I64, I64,
+                                                      I64, I64, I]
+            lib.la_oracle_backward_recurrent.argtypes = [P, P, P, P, I, P, P, P, P, I64, I64, I64,
+                                                         I64, I64, I]
             for f in ("la_oracle_masked", "la_oracle_recurrent", "la_oracle_recurrent_sampled",
-                      "la_oracle_blocked", "la_oracle_decode_step", "la_oracle_max_threads"):
+                      "la_oracle_blocked", "la_oracle_decode_step", "la_oracle_max_threads",
+                      "la_oracle_masked_anticausal", "la_oracle_recurrent_anticausal",
+                      "la_oracle_backward_masked", "la_oracle_backward_recurrent"):
                 getattr(lib, f).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -162,6 +174,57 @@ def decode_step(q, k, v, slopes, state, threads: int = 0) -> np.ndarray:
     _check(_load().la_oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(s), _ptr(state),
                                          _ptr(out), B, H, D, E, threads), "la_oracle_decode_step")
     return out
+
+
+def masked_anticausal(q, k, v, slopes, threads: int = 0) -> np.ndarray:
+    """o_t = sum_{s >= t} exp(-lambda (s - t)) (q_t . k_s) v_s, term by term."""
+    q, k, v, dt = _inputs(q, k, v)
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    s = _slopes(slopes, H)
+    out = np.empty((B, H, N, E), dtype=np.float64)
+    _check(_load().la_oracle_masked_anticausal(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(s), _ptr(out),
+                                               B, H, N, D, E, threads),
+           "la_oracle_masked_anticausal")
+    return out
+
+
+def recurrent_anticausal(q, k, v, slopes, s0=None, return_state: bool = False, threads: int = 0):
+    """The anti-causal sum as a recurrence run from the last token down; s0 is
+    the state after the last token, the returned state the one at token 0."""
+    q, k, v, dt = _inputs(q, k, v)
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    s = _slopes(slopes, H)
+    out = np.empty((B, H, N, E), dtype=np.float64)
+    s0a = None if s0 is None else np.ascontiguousarray(s0, dtype=np.float64).reshape(B, H, D, E)
+    sf = np.empty((B, H, D, E), dtype=np.float64) if return_state else None
+    _check(_load().la_oracle_recurrent_anticausal(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(s),
+                                                  _ptr(s0a), _ptr(sf), _ptr(out), B, H, N, D, E,
+                                                  threads), "la_oracle_recurrent_anticausal")
+    return (out, sf) if return_state else out
+
+
+def backward(q, k, v, dout, slopes, form: str = "recurrent", threads: int = 0):
+    """Gradients (dq, dk, dv) of L = sum_t dout_t . o_t (float64), as recurrences
+    (form="recurrent", O(N D E)) or as the written-out sums (form="masked")."""
+    q, k, v, dt = _inputs(q, k, v)
+    g = np.ascontiguousarray(dout)
+    if g.dtype != q.dtype:
+        raise TypeError("dout must have the dtype of q, k, v")
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    if g.shape != (B, H, N, E):
+        raise ValueError("dout must be [B,H,N,E]")
+    s = _slopes(slopes, H)
+    dq = np.empty((B, H, N, D), dtype=np.float64)
+    dk = np.empty((B, H, N, D), dtype=np.float64)
+    dv = np.empty((B, H, N, E), dtype=np.float64)
+    fn = {"recurrent": _load().la_oracle_backward_recurrent,
+          "masked": _load().la_oracle_backward_masked}[form]
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), dt, _ptr(s), _ptr(dq), _ptr(dk), _ptr(dv),
+              B, H, N, D, E, threads), f"la_oracle_backward_{form}")
+    return dq, dk, dv
 
 
 def max_threads() -> int:

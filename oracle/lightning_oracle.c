@@ -29,6 +29,20 @@
  *   la_oracle_recurrent_sampled  the recurrence, emitting o_t only at the
  *                        given positions (for sequences too long to store).
  *   la_oracle_decode_step one recurrent step on a given state, in place.
+ *
+ * Reverse time and gradients (for the backward pass of training; the pages
+ * train with 1M-token contexts, abstract and "MiniMax-01" blog):
+ *   la_oracle_masked_anticausal / la_oracle_recurrent_anticausal
+ *        o_t = sum_{s >= t} exp(-lambda (s - t)) (q_t . k_s) v_s, the same sum
+ *        with time reversed (definition, and the recurrence run from t = N-1
+ *        down: S_t = gamma S_{t+1} + k_t^T v_t, o_t = q_t S_t).
+ *   la_oracle_backward_masked / la_oracle_backward_recurrent
+ *        the gradients of L = sum_t dout_t . o_t:
+ *          dq_t = sum_{s <= t} g^(t-s) (dout_t . v_s) k_s
+ *          dk_s = sum_{t >= s} g^(t-s) (dout_t . v_s) q_t
+ *          dv_s = sum_{t >= s} g^(t-s) (q_t . k_s) dout_t      (g = gamma)
+ *        (the derivative of the masked sum written out term by term, and the
+ *        same sums as recurrences: forward for dq, backward in time for dk, dv).
  */
 #include <math.h>
 #include <stdint.h>
@@ -289,6 +303,202 @@ int la_oracle_decode_step(const void* q, const void* k, const void* v, int dtype
       double qd = in_at(q, bh * D + d, dtype);
       for (int64_t e = 0; e < E; ++e) o[e] += qd * S[d * E + e];
     }
+  }
+  return 0;
+}
+
+/* Anti-causal masked sum: the definition with time reversed, term by term. */
+int la_oracle_masked_anticausal(const void* q, const void* k, const void* v, int dtype,
+                                const float* slopes, double* out, int64_t B, int64_t H, int64_t N,
+                                int64_t D, int64_t E, int nthreads) {
+  int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
+  if (rc) return rc;
+  set_threads(nthreads);
+  int64_t BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    double lam = (double)slopes[bh % H];
+    double* Q = (double*)malloc(sizeof(double) * (size_t)(N * D + 1));
+    double* K = (double*)malloc(sizeof(double) * (size_t)(N * D + 1));
+    double* V = (double*)malloc(sizeof(double) * (size_t)(N * E + 1));
+    in_row(Q, q, bh * N * D, N * D, dtype);
+    in_row(K, k, bh * N * D, N * D, dtype);
+    in_row(V, v, bh * N * E, N * E, dtype);
+    double* O = out + bh * N * E;
+    for (int64_t t = 0; t < N; ++t) {
+      for (int64_t e = 0; e < E; ++e) O[t * E + e] = 0.0;
+      for (int64_t s = t; s < N; ++s) {
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += Q[t * D + d] * K[s * D + d];
+        double w = exp(-lam * (double)(s - t)) * dot;
+        for (int64_t e = 0; e < E; ++e) O[t * E + e] += w * V[s * E + e];
+      }
+    }
+    free(Q);
+    free(K);
+    free(V);
+  }
+  return 0;
+}
+
+/*
+ * Anti-causal recurrence S_t = gamma S_{t+1} + k_t^T v_t for t = N-1 .. 0,
+ * o_t = q_t S_t.  s0 (nullable) is S_N (zero if NULL); s_final (nullable)
+ * receives S_0 (or s0 when N == 0).
+ */
+int la_oracle_recurrent_anticausal(const void* q, const void* k, const void* v, int dtype,
+                                   const float* slopes, const double* s0, double* s_final,
+                                   double* out, int64_t B, int64_t H, int64_t N, int64_t D,
+                                   int64_t E, int nthreads) {
+  int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
+  if (rc) return rc;
+  set_threads(nthreads);
+  int64_t BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    double gamma = exp(-(double)slopes[bh % H]);
+    double* S = (double*)calloc((size_t)(D * E), sizeof(double));
+    double* qt = (double*)malloc(sizeof(double) * (size_t)D);
+    double* kt = (double*)malloc(sizeof(double) * (size_t)D);
+    double* vt = (double*)malloc(sizeof(double) * (size_t)E);
+    if (s0) memcpy(S, s0 + bh * D * E, sizeof(double) * (size_t)(D * E));
+    double* O = out + bh * N * E;
+    for (int64_t t = N - 1; t >= 0; --t) {
+      in_row(qt, q, (bh * N + t) * D, D, dtype);
+      in_row(kt, k, (bh * N + t) * D, D, dtype);
+      in_row(vt, v, (bh * N + t) * E, E, dtype);
+      for (int64_t d = 0; d < D; ++d)
+        for (int64_t e = 0; e < E; ++e) S[d * E + e] = gamma * S[d * E + e] + kt[d] * vt[e];
+      for (int64_t e = 0; e < E; ++e) O[t * E + e] = 0.0;
+      for (int64_t d = 0; d < D; ++d)
+        for (int64_t e = 0; e < E; ++e) O[t * E + e] += qt[d] * S[d * E + e];
+    }
+    if (s_final) memcpy(s_final + bh * D * E, S, sizeof(double) * (size_t)(D * E));
+    free(S);
+    free(qt);
+    free(kt);
+    free(vt);
+  }
+  return 0;
+}
+
+static int bad_grads(const void* dout, const double* dq, const double* dk, const double* dv) {
+  return (!dout || !dq || !dk || !dv) ? 1 : 0;
+}
+
+/* Gradients of L = sum_t dout_t . o_t, each sum written out term by term. */
+int la_oracle_backward_masked(const void* q, const void* k, const void* v, const void* dout,
+                              int dtype, const float* slopes, double* dq, double* dk, double* dv,
+                              int64_t B, int64_t H, int64_t N, int64_t D, int64_t E,
+                              int nthreads) {
+  int rc = bad_args(q, k, v, slopes, dq, B, H, N, D, E);
+  if (rc) return rc;
+  if (bad_grads(dout, dq, dk, dv)) return 1;
+  set_threads(nthreads);
+  int64_t BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    double lam = (double)slopes[bh % H];
+    double* Q = (double*)malloc(sizeof(double) * (size_t)(N * D + 1));
+    double* K = (double*)malloc(sizeof(double) * (size_t)(N * D + 1));
+    double* V = (double*)malloc(sizeof(double) * (size_t)(N * E + 1));
+    double* G = (double*)malloc(sizeof(double) * (size_t)(N * E + 1));
+    in_row(Q, q, bh * N * D, N * D, dtype);
+    in_row(K, k, bh * N * D, N * D, dtype);
+    in_row(V, v, bh * N * E, N * E, dtype);
+    in_row(G, dout, bh * N * E, N * E, dtype);
+    double* dQ = dq + bh * N * D;
+    double* dK = dk + bh * N * D;
+    double* dV = dv + bh * N * E;
+    for (int64_t x = 0; x < N * D; ++x) dQ[x] = dK[x] = 0.0;
+    for (int64_t x = 0; x < N * E; ++x) dV[x] = 0.0;
+    for (int64_t t = 0; t < N; ++t)
+      for (int64_t s = 0; s <= t; ++s) {
+        double w = exp(-lam * (double)(t - s));
+        double gv = 0.0, qk = 0.0;
+        for (int64_t e = 0; e < E; ++e) gv += G[t * E + e] * V[s * E + e];
+        for (int64_t d = 0; d < D; ++d) qk += Q[t * D + d] * K[s * D + d];
+        for (int64_t d = 0; d < D; ++d) {
+          dQ[t * D + d] += w * gv * K[s * D + d];
+          dK[s * D + d] += w * gv * Q[t * D + d];
+        }
+        for (int64_t e = 0; e < E; ++e) dV[s * E + e] += w * qk * G[t * E + e];
+      }
+    free(Q);
+    free(K);
+    free(V);
+    free(G);
+  }
+  return 0;
+}
+
+/*
+ * The same gradients as recurrences (O(N D E)):
+ *   T_t = gamma T_{t-1} + v_t^T k_t (E x D),  dq_t = dout_t T_t        (t up)
+ *   U_t = gamma U_{t+1} + dout_t^T q_t (E x D), dk_t = v_t U_t         (t down)
+ *   W_t = gamma W_{t+1} + q_t^T dout_t (D x E), dv_t = k_t W_t         (t down)
+ */
+int la_oracle_backward_recurrent(const void* q, const void* k, const void* v, const void* dout,
+                                 int dtype, const float* slopes, double* dq, double* dk,
+                                 double* dv, int64_t B, int64_t H, int64_t N, int64_t D,
+                                 int64_t E, int nthreads) {
+  int rc = bad_args(q, k, v, slopes, dq, B, H, N, D, E);
+  if (rc) return rc;
+  if (bad_grads(dout, dq, dk, dv)) return 1;
+  set_threads(nthreads);
+  int64_t BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    double gamma = exp(-(double)slopes[bh % H]);
+    double* T = (double*)calloc((size_t)(E * D), sizeof(double));
+    double* qt = (double*)malloc(sizeof(double) * (size_t)D);
+    double* kt = (double*)malloc(sizeof(double) * (size_t)D);
+    double* vt = (double*)malloc(sizeof(double) * (size_t)E);
+    double* gt = (double*)malloc(sizeof(double) * (size_t)E);
+    double* dQ = dq + bh * N * D;
+    double* dK = dk + bh * N * D;
+    double* dV = dv + bh * N * E;
+    for (int64_t t = 0; t < N; ++t) {  /* dq, forward in time */
+      in_row(kt, k, (bh * N + t) * D, D, dtype);
+      in_row(vt, v, (bh * N + t) * E, E, dtype);
+      in_row(gt, dout, (bh * N + t) * E, E, dtype);
+      for (int64_t e = 0; e < E; ++e)
+        for (int64_t d = 0; d < D; ++d) T[e * D + d] = gamma * T[e * D + d] + vt[e] * kt[d];
+      for (int64_t d = 0; d < D; ++d) {
+        double acc = 0.0;
+        for (int64_t e = 0; e < E; ++e) acc += gt[e] * T[e * D + d];
+        dQ[t * D + d] = acc;
+      }
+    }
+    double* U = T;  /* E x D, reused */
+    double* W = (double*)calloc((size_t)(D * E), sizeof(double));
+    for (int64_t x = 0; x < E * D; ++x) U[x] = 0.0;
+    for (int64_t t = N - 1; t >= 0; --t) {  /* dk, dv, backward in time */
+      in_row(qt, q, (bh * N + t) * D, D, dtype);
+      in_row(kt, k, (bh * N + t) * D, D, dtype);
+      in_row(vt, v, (bh * N + t) * E, E, dtype);
+      in_row(gt, dout, (bh * N + t) * E, E, dtype);
+      for (int64_t e = 0; e < E; ++e)
+        for (int64_t d = 0; d < D; ++d) U[e * D + d] = gamma * U[e * D + d] + gt[e] * qt[d];
+      for (int64_t d = 0; d < D; ++d)
+        for (int64_t e = 0; e < E; ++e) W[d * E + e] = gamma * W[d * E + e] + qt[d] * gt[e];
+      for (int64_t d = 0; d < D; ++d) {
+        double acc = 0.0;
+        for (int64_t e = 0; e < E; ++e) acc += vt[e] * U[e * D + d];
+        dK[t * D + d] = acc;
+      }
+      for (int64_t e = 0; e < E; ++e) {
+        double acc = 0.0;
+        for (int64_t d = 0; d < D; ++d) acc += kt[d] * W[d * E + e];
+        dV[t * E + e] = acc;
+      }
+    }
+    free(T);
+    free(W);
+    free(qt);
+    free(kt);
+    free(vt);
+    free(gt);
   }
   return 0;
 }
