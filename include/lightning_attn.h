@@ -176,6 +176,38 @@ int lightning_attn_decode(const void* q, const void* k, const void* v,
                           int B, int H, int D, int E, void* stream);
 
 /*
+ * Anti-causal prefill: o_t = sum_{s >= t} exp(-lambda_h (s - t)) (q_t . k_s) v_s,
+ * the same operation with time reversed (needed by the backward pass below).
+ * init_state is the state after the last token (zero if NULL); final_state
+ * receives the state at token 0.  Otherwise as lightning_attn_fwd_ex (layouts
+ * [B][H][N][*], bf16 q, k, v, fp32 out, D, E in {64, 128}, chunk, errors).
+ * The pages state only the causal operator; reversal is the plain reading of
+ * what its gradients need.
+ */
+int lightning_attn_fwd_anticausal(const void* q, const void* k, const void* v, const float* slopes,
+                                  const float* init_state, float* final_state, float* out, int B,
+                                  int H, int N, int D, int E, int chunk, void* stream);
+
+/*
+ * Backward pass of lightning_attn_fwd for training (the abstract: contexts of
+ * 1M tokens in training): given dout = dL/d out (bf16 [B][H][N][E]), writes
+ * the gradients with respect to the inputs, fp32:
+ *   dq_t = sum_{s <= t} g^(t-s) (dout_t . v_s) k_s      dq [B][H][N][D]
+ *   dk_s = sum_{t >= s} g^(t-s) (dout_t . v_s) q_t      dk [B][H][N][D]
+ *   dv_s = sum_{t >= s} g^(t-s) (q_t . k_s) dout_t      dv [B][H][N][E]
+ * (g = exp(-lambda_h); zero initial state; the slopes are not differentiated).
+ * dq is the causal operator applied to (dout, v, k); dk and dv are the
+ * anti-causal operator applied to (v, dout, q) and (k, q, dout): three
+ * launches of the tensor-core kernel on `stream`.  bf16 inputs as for the
+ * forward pass, D, E in {64, 128}; dq, dk, dv 16-byte aligned and not
+ * overlapping the inputs or each other (not checked).  Errors as
+ * lightning_attn_fwd (the first failing launch's code).
+ */
+int lightning_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
+                       const float* slopes, float* dq, float* dk, float* dv, int B, int H, int N,
+                       int D, int E, void* stream);
+
+/*
  * Fault-injection hook for testing the bounded device-side waits (an interface
  * for tests; the pages have no counterpart).  Runs the chunked bf16 prefill
  * (D = E = 128, chunk a multiple of 128 with N > chunk) but hands out work

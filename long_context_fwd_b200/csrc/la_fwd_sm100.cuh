@@ -307,7 +307,15 @@ __device__ __forceinline__ void tile_store(const CUtensorMap* map, const void* s
 // ---------------------------------------------------------------------------
 // Producer: one thread issues every TMA load.
 // ---------------------------------------------------------------------------
-template <int RANK>
+// REV (anti-causal runs): work items and blocks are in reversed token order
+// tau = N - 1 - t; the tile of tau-block [tb, tb + 128) is tokens
+// [N - tb - 128, N - tb), loaded in increasing token order (a negative start
+// row reads zeros), so a tile row r holds local reversed index 127 - r.
+__device__ __forceinline__ int tile_row(const Params& p, int tb, bool rev) {
+  return rev ? p.N - tb - BLK : tb;
+}
+
+template <int RANK, bool REV>
 __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
                          const CUtensorMap* tk, const CUtensorMap* tv) {
   const uint64_t pol_first = policy_evict_first();
@@ -372,7 +380,7 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
         if (b < P1_SLOTS) ok = ring_released(slot);  // first use in this item
         if (ok && use >= 1) ok = wait_bar(c, p, B_P1E + slot, (use - 1) & 1u);
         if (!ok) break;
-        const int row = it.t0 + b * BLK;
+        const int row = tile_row(p, it.t0 + b * BLK, REV);
         uint8_t* dst = c.sm + p1_base(slot);
         uint64_t* full = &c.bar[B_P1F + slot];
         mbar_arrive_expect_tx(full, 2 * TILE);
@@ -390,7 +398,7 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
       pairs_pending = false;
     }
     for (int n = 0; n < (it.p2 ? it.nb : 0) && ok; ++n) {
-      const int row = it.t0 + n * BLK;
+      const int row = tile_row(p, it.t0 + n * BLK, REV);
       ok = load(B_QF, B_QE, OFF_Q, q_it, tq, 0, row, it.seq, hh, bb, pol_first) &&
            load(B_KF, B_KE, OFF_K, k_it, tk, 1, row, it.seq, hh, bb, pol_first) &&
            load(B_VF, B_VE, OFF_V, v_it, tv, 2, row, it.seq, hh, bb, pol_first);
@@ -520,6 +528,7 @@ __device__ void mma_issuer(const Ctx& c, const Params& p) {
 // ---------------------------------------------------------------------------
 // Group X: decay-causal mask and the in-place operand decays.
 // ---------------------------------------------------------------------------
+template <bool REV>
 __device__ void group_x(const Ctx& c, const Params& p) {
   const uint32_t t = threadIdx.x - 32u * X_WARP0;  // 0..255
   const uint32_t warp = t >> 5;
@@ -548,7 +557,8 @@ __device__ void group_x(const Ctx& c, const Params& p) {
       for (int b = 0; b < it.nb && ok; ++b) {
         const uint32_t slot = p1_it % P1_SLOTS;
         if (!cwait(c, p, B_P1F + slot, (p1_it / P1_SLOTS) & 1u)) { ok = false; break; }
-        const int jc = b * BLK + static_cast<int>(r);
+        // reversed chunk-local index of this tile row (REV: row r is 127 - r)
+        const int jc = b * BLK + static_cast<int>(REV ? 127u - r : r);
         const float f = jc < it.Lc ? expf(-lam * static_cast<float>(it.Lc - 1 - jc)) : 0.f;
         scale_row(c.sbase + p1_base(slot) + hf * PLANE + r * 128u, r, f);
         fence_proxy_async_smem();
@@ -571,7 +581,10 @@ __device__ void group_x(const Ctx& c, const Params& p) {
       // have zero scores (zero-filled Q), so they give zero P as well.  In the
       // quarter with every column above every row (hf = 1, rows < 64) P is 0.
       uint32_t pk[32];
-      if (hf == 1 && (warp & 3u) < 2) {
+      // causal: P_rc = S_rc gamma^(r-c) for c <= r; anti-causal (rows in
+      // reversed order): P_rc = S_rc gamma^(c-r) for c >= r.  The quadrant
+      // where the condition fails for every (r, c) is zero.
+      if (REV ? (hf == 0 && (warp & 3u) >= 2) : (hf == 1 && (warp & 3u) < 2)) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = 0u;
       } else {
@@ -579,18 +592,29 @@ __device__ void group_x(const Ctx& c, const Params& p) {
         for (uint32_t half = 0; half < 2; ++half) {
           uint32_t sc[32];
           tmem_ld32(t_s + half * 32u, sc);
-          const uint32_t u0 = gtab + 4u * (hf * 64u + half * 32u + 127u - r);
           tmem_wait_ld();
+          if (REV) {
+            const uint32_t u0 = gtab + 4u * (r + 127u - hf * 64u - half * 32u);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[16 * half + i] = pack_bf16x2(__uint_as_float(sc[2 * i]) * lds32f(u0 + 8u * i),
-                                            __uint_as_float(sc[2 * i + 1]) * lds32f(u0 + 8u * i + 4u));
+            for (int i = 0; i < 16; ++i)
+              pk[16 * half + i] =
+                  pack_bf16x2(__uint_as_float(sc[2 * i]) * lds32f(u0 - 8u * i),
+                              __uint_as_float(sc[2 * i + 1]) * lds32f(u0 - 8u * i - 4u));
+          } else {
+            const uint32_t u0 = gtab + 4u * (hf * 64u + half * 32u + 127u - r);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[16 * half + i] =
+                  pack_bf16x2(__uint_as_float(sc[2 * i]) * lds32f(u0 + 8u * i),
+                              __uint_as_float(sc[2 * i + 1]) * lds32f(u0 + 8u * i + 4u));
+          }
         }
       }
       tmem_st32(t_s, pk);
       // gamma^(r+1) Q (bf16) into the S buffer's free columns; the Q tile is then dead
       {
-        const float fq = lds32f(gtab + 4u * (127u - r)) * lds32f(gtab + 4u * 126u);
+        // gamma^(i+1) for the (reversed, if REV) local index i of row r
+        const float fq = lds32f(gtab + 4u * (REV ? r : 127u - r)) * lds32f(gtab + 4u * 126u);
         const uint32_t qrow = c.sbase + OFF_Q + qs * TILE + hf * PLANE + r * 128u;
         uint32_t qv[32];
 #pragma unroll
@@ -605,7 +629,9 @@ __device__ void group_x(const Ctx& c, const Params& p) {
         tmem_st32(t_s + 32u, qv);
       }
       // gamma^(len-1-r) K (0 past len) in place
-      const float fk = lds32f(gtab + 4u * (128u - static_cast<uint32_t>(len) + r));
+      // gamma^(len-1-j) for the local index j of row r (0 past len)
+      const float fk = lds32f(gtab + 4u * (REV ? 255u - static_cast<uint32_t>(len) - r
+                                               : 128u - static_cast<uint32_t>(len) + r));
       scale_row(c.sbase + OFF_K + ks * TILE + hf * PLANE + r * 128u, r, fk);
       fence_proxy_async_smem();
       tmem_wait_st();
@@ -670,7 +696,7 @@ __device__ __forceinline__ void st_scan32(float* base, uint32_t r, uint32_t hf, 
                        __uint_as_float(x[4 * i + 2]), __uint_as_float(x[4 * i + 3])));
 }
 
-template <int RANK>
+template <int RANK, bool REV>
 __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
   const uint32_t t = threadIdx.x - 32u * Y_WARP0;  // 0..127
   const uint32_t r = t;                            // TMEM lane / tile row
@@ -861,7 +887,30 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
       tc_fence_after();
       const uint32_t vtile = c.sbase + OFF_V + vs * TILE;
       const uint8_t* vtile_g = c.sm + OFF_V + vs * TILE;
-      const int row = it.t0 + n * BLK;
+      const int row = tile_row(p, it.t0 + n * BLK, REV);
+      if (REV && row < 0) {
+        // The block holding token 0 of an anti-causal run starts at a
+        // negative row, where a TMA store may not start: plain stores of the
+        // rows that exist, straight from TMEM.  The V slot is not needed.
+        const int tok = row + static_cast<int>(r);
+        float* dst = tok >= 0 ? p.out + (it.seq / p.H) * p.ostride[0] + (it.seq % p.H) * p.ostride[1] +
+                                     static_cast<int64_t>(tok) * p.ostride[2]
+                              : nullptr;
+#pragma unroll 1
+        for (uint32_t qq = 0; qq < 4; ++qq) {
+          uint32_t o[32];
+          tmem_ld32(t_o + 32u * qq, o);
+          tmem_wait_ld();
+          if (dst && 32 * static_cast<int>(qq) < p.E) st_global32(dst + 32 * qq, o);
+        }
+        tc_fence_before();
+        warp_arrive(&c.bar[B_O_EMPTY]);
+        if (leader) mbar_arrive(&c.bar[B_VE + vs]);
+        if (leader) LA_TRACE_EVENT(14, g);
+        ++v_it;
+        ++gb;
+        continue;
+      }
       uint32_t o0[32], o1[32];
       tmem_ld32(t_o, o0);
       tmem_ld32(t_o + 32u, o1);
@@ -913,7 +962,8 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
 // 14 warps on 4 SM sub-partitions (16K registers each, at most 4 warps on one)
 // leave up to 128 registers per thread.
 // RANK: 3 for contiguous head-major q, k, v, out; 4 for strided layouts.
-template <int RANK>
+// REV: anti-causal (o_t sums s >= t), the same blocked form in reversed time.
+template <int RANK, bool REV>
 __global__ void __launch_bounds__(THREADS, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
@@ -978,14 +1028,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   c.tmem = c.misc[0];
 
   if (warp == PRODUCER_WARP) {
-    if (lane_id() == 0) producer<RANK>(c, p, &tq, &tk, &tv);
+    if (lane_id() == 0) producer<RANK, REV>(c, p, &tq, &tk, &tv);
   } else if (warp == MMA_WARP) {
     if (lane_id() == 0) mma_issuer(c, p);
     __syncwarp();
   } else if (warp < Y_WARP0) {
-    group_x(c, p);
+    group_x<REV>(c, p);
   } else {
-    group_y<RANK>(c, p, &to);
+    group_y<RANK, REV>(c, p, &to);
   }
 
   tc_fence_before();

@@ -34,6 +34,8 @@ struct Params {
   int cslot[4];               // q, k, v, out tensor maps: where t, h, b sit (make_tmap_4d)
   int D, E;                   // the caller's head dimensions (64 or 128; tiles are 128 wide,
                               // the tensor maps zero-fill the columns past D or E)
+  float* out;                 // the output and its element strides {b, h, t}, for rows that
+  long long ostride[3];       // are stored without TMA (anti-causal runs, first block)
   unsigned long long wait_limit_ns;
 };
 

@@ -250,10 +250,11 @@ bool build_maps(const void* q, const void* k, const void* v, const float* out, i
 
 // Launches the prefill kernel for the map rank (sets the shared-memory
 // attribute on every call: it belongs to the current device's context).
-int launch_fwd(int rank, int grid, cudaStream_t stream, const CUtensorMap& tq,
+int launch_fwd(int rank, bool rev, int grid, cudaStream_t stream, const CUtensorMap& tq,
                const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                const la::fwd::Params& p) {
-  auto kern = rank == 3 ? la::fwd::fwd_bf16_kernel<3> : la::fwd::fwd_bf16_kernel<4>;
+  auto kern = rank == 3 ? (rev ? la::fwd::fwd_bf16_kernel<3, true> : la::fwd::fwd_bf16_kernel<3, false>)
+                        : (rev ? la::fwd::fwd_bf16_kernel<4, true> : la::fwd::fwd_bf16_kernel<4, false>);
   const cudaError_t attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::fwd::SMEM_BYTES);
   if (attr != cudaSuccess) return cuda_fail(attr);
@@ -264,7 +265,8 @@ int launch_fwd(int rank, int grid, cudaStream_t stream, const CUtensorMap& tq,
 int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slopes,
                   const float* init_state, float* final_state, float* out, int B, int H, int N,
                   int D, int E, int chunk, void* stream_ptr, const Strides* strides = nullptr,
-                  int first_chunk = 0, unsigned long long wait_limit_ns = kWaitLimitNs) {
+                  bool reverse = false, int first_chunk = 0,
+                  unsigned long long wait_limit_ns = kWaitLimitNs) {
   if (!q || !k || !v || !slopes || !out) return LA_ERR_NULL;
   if (!dims_ok(B, H, N, D, E)) return LA_ERR_SHAPE;
   if ((D != 64 && D != 128) || (E != 64 && E != 128)) return LA_ERR_UNSUPPORTED;
@@ -285,6 +287,8 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   int rank = 3;
   if (!build_maps(q, k, v, out, B, H, N, D, E, st, &tq, &tk, &tv, &to, p, &rank))
     return LA_ERR_CUDA;
+  p.out = out;
+  for (int j = 0; j < 3; ++j) p.ostride[j] = st.s[3][j];
 
   p.slopes = slopes;
   p.init_state = init_state;
@@ -309,7 +313,7 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
     set_scratch(pl, scratch, p);
   }
 
-  int rc = launch_fwd(rank, pl.grid, stream, tq, tk, tv, to, p);
+  int rc = launch_fwd(rank, reverse, pl.grid, stream, tq, tk, tv, to, p);
   if (scratch) {
     const cudaError_t e = cudaFreeAsync(scratch, stream);
     if (e != cudaSuccess && rc == LA_OK) rc = cuda_fail(e);
@@ -393,7 +397,7 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
     if (e != cudaSuccess) return cuda_fail(e);
     set_scratch(pl, scratch, p);
   }
-  return launch_fwd(rank, pl.grid, stream, tq, tk, tv, to, p);
+  return launch_fwd(rank, false, pl.grid, stream, tq, tk, tv, to, p);
 }
 
 template <int D, int E>
@@ -447,13 +451,37 @@ int lightning_attn_fwd_strided(const void* q, const void* k, const void* v, cons
                        stream, &st);
 }
 
+int lightning_attn_fwd_anticausal(const void* q, const void* k, const void* v, const float* slopes,
+                                  const float* init_state, float* final_state, float* out, int B,
+                                  int H, int N, int D, int E, int chunk, void* stream) {
+  return fwd_bf16_impl(q, k, v, slopes, init_state, final_state, out, B, H, N, D, E, chunk,
+                       stream, nullptr, /*reverse=*/true);
+}
+
+int lightning_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
+                       const float* slopes, float* dq, float* dk, float* dv, int B, int H, int N,
+                       int D, int E, void* stream) {
+  if (!dout || !dq || !dk || !dv) return LA_ERR_NULL;
+  // dq_t = sum_{s<=t} g^(t-s) (dout_t . v_s) k_s: the causal operator on (dout, v, k)
+  int rc = fwd_bf16_impl(dout, v, k, slopes, nullptr, nullptr, dq, B, H, N, E, D, 0, stream);
+  if (rc != LA_OK) return rc;
+  // dk_s = sum_{t>=s} g^(t-s) (v_s . dout_t) q_t: the anti-causal operator on (v, dout, q)
+  rc = fwd_bf16_impl(v, dout, q, slopes, nullptr, nullptr, dk, B, H, N, E, D, 0, stream, nullptr,
+                     true);
+  if (rc != LA_OK) return rc;
+  // dv_s = sum_{t>=s} g^(t-s) (k_s . q_t) dout_t: the anti-causal operator on (k, q, dout)
+  return fwd_bf16_impl(k, q, dout, slopes, nullptr, nullptr, dv, B, H, N, D, E, 0, stream, nullptr,
+                       true);
+}
+
 int lightning_attn_fault_test_scan_stall(const void* q, const void* k, const void* v,
                                          const float* slopes, float* out, int B, int H, int N,
                                          int chunk, unsigned int wait_limit_ms, void* stream) {
   if (chunk <= 0 || N <= chunk) return LA_ERR_SHAPE;  // needs at least two chunks
   if (wait_limit_ms == 0 || wait_limit_ms > 10000) return LA_ERR_SHAPE;
   return fwd_bf16_impl(q, k, v, slopes, nullptr, nullptr, out, B, H, N, 128, 128, chunk, stream,
-                       /*strides=*/nullptr, /*first_chunk=*/1, 1000000ull * wait_limit_ms);
+                       /*strides=*/nullptr, /*reverse=*/false, /*first_chunk=*/1,
+                       1000000ull * wait_limit_ms);
 }
 
 int lightning_attn_fwd_noalloc(const void* q, const void* k, const void* v, const float* slopes,

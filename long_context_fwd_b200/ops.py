@@ -36,6 +36,8 @@ SIGNATURES = {
     "lightning_attn_last_cuda_error": [],
     "lightning_attn_device_status": [_P, _I],
     "lightning_attn_fwd_plan": [_I, _I, _I, _I, _I, _P, _P, _I, _P],
+    "lightning_attn_fwd_anticausal": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P],
+    "lightning_attn_bwd": [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P],
     "lightning_attn_fwd_strided": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P,
                                    _I, _P],
 }
@@ -170,6 +172,52 @@ def fwd_strided(q, k, v, slopes, out, *, init_state=None, final_state=None, chun
         int(chunk), _stream_handle(stream))
     _check("lightning_attn_fwd_strided", rc)
     return out
+
+
+def fwd_anticausal(q, k, v, slopes, out=None, *, init_state=None, final_state=None,
+                   chunk: int = 0, stream=None) -> torch.Tensor:
+    """Anti-causal prefill, o_t = sum_{s >= t} g^(s-t) (q_t . k_s) v_s (shapes as fwd)."""
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    _need(q, "q", torch.bfloat16, (B, H, N, D))
+    _need(k, "k", torch.bfloat16, (B, H, N, D))
+    _need(v, "v", torch.bfloat16, (B, H, N, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    if out is None:
+        out = torch.empty((B, H, N, E), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, H, N, E))
+    for name, st in (("init_state", init_state), ("final_state", final_state)):
+        if st is not None:
+            _need(st, name, torch.float32, (B, H, D, E))
+    rc = lib().lightning_attn_fwd_anticausal(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), slopes.data_ptr(),
+        None if init_state is None else init_state.data_ptr(),
+        None if final_state is None else final_state.data_ptr(),
+        out.data_ptr(), B, H, N, D, E, int(chunk), _stream_handle(stream))
+    _check("lightning_attn_fwd_anticausal", rc)
+    return out
+
+
+def bwd(q, k, v, dout, slopes, dq=None, dk=None, dv=None, *, stream=None):
+    """Backward pass: bf16 q, k [B,H,N,D], v, dout [B,H,N,E] -> fp32 (dq, dk, dv)."""
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    _need(q, "q", torch.bfloat16, (B, H, N, D))
+    _need(k, "k", torch.bfloat16, (B, H, N, D))
+    _need(v, "v", torch.bfloat16, (B, H, N, E))
+    _need(dout, "dout", torch.bfloat16, (B, H, N, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    dq = torch.empty((B, H, N, D), dtype=torch.float32, device=q.device) if dq is None else dq
+    dk = torch.empty((B, H, N, D), dtype=torch.float32, device=q.device) if dk is None else dk
+    dv = torch.empty((B, H, N, E), dtype=torch.float32, device=q.device) if dv is None else dv
+    _need(dq, "dq", torch.float32, (B, H, N, D))
+    _need(dk, "dk", torch.float32, (B, H, N, D))
+    _need(dv, "dv", torch.float32, (B, H, N, E))
+    rc = lib().lightning_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
+                                  slopes.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                  B, H, N, D, E, _stream_handle(stream))
+    _check("lightning_attn_bwd", rc)
+    return dq, dk, dv
 
 
 def fwd_noalloc(q, k, v, slopes, out=None, *, chunk: int = 0, stream=None) -> torch.Tensor:

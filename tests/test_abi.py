@@ -127,3 +127,14 @@ def test_strided_validation(lib):
     assert f(*args(ok, ok, ok, bad_o)) == LA_ERR_ALIGN
     assert f(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 4, 64, 32, 128, ok, ok, ok, ok_o, 0,
              None) == LA_ERR_UNSUPPORTED
+
+
+def test_backward_and_anticausal_validation(lib):
+    f = lib.lightning_attn_bwd
+    assert f(FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 128, 128, None) == LA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 96, 128, None) == LA_ERR_UNSUPPORTED
+    g = lib.lightning_attn_fwd_anticausal
+    assert g(None, FAKE, FAKE, FAKE, None, None, FAKE, 1, 1, 8, 128, 128, 0, None) == LA_ERR_NULL
+    assert g(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 1, 8, 128, 128, 100, None) == LA_ERR_SHAPE
