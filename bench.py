@@ -108,6 +108,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the end-to-end leg")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="0 skips the CPU baseline")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--backward-steps", type=int, default=20,
+                    help="steps of the backward-pass leg (0 skips it)")
     return ap.parse_args()
 
 
@@ -327,6 +329,45 @@ def bench_decode(args, dist, dev):
             "finite": finite, "workload": w.name, "tokens": w.B}
 
 
+def bench_backward(args, dist, w, dev):
+    """The backward pass (dq, dk, dv from dout) on the prefill workload's shapes:
+    three launches of the tensor-core kernel per step (dq causal, dk and dv
+    anti-causal), inputs resident on the device."""
+    import torch
+    from long_context_fwd_b200 import inputs as I
+    from long_context_fwd_b200 import ops
+
+    q, k, v = I.device_prefill_inputs(w, dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(98765)
+    dout = torch.randn((w.B, w.H, w.N, w.E), generator=g, device=dev).to(torch.bfloat16)
+    sl = torch.from_numpy(I.slopes_for(w)).to(dev)
+    dq = torch.empty((w.B, w.H, w.N, w.D), dtype=torch.float32, device=dev)
+    dk = torch.empty_like(dq)
+    dv = torch.empty((w.B, w.H, w.N, w.E), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        ops.bwd(q, k, v, dout, sl, dq, dk, dv)
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0, "device-side wait timed out during warm-up"
+    dist.barrier()
+    steps = args.backward_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_host0 = time.time()
+    e0.record(stream)
+    for _ in range(steps):
+        ops.bwd(q, k, v, dout, sl, dq, dk, dv)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.time()
+    dist.barrier()
+    ms = dist.max(e0.elapsed_time(e1)) / steps
+    status = ops.device_status(reset=True)
+    del q, k, v, dout, dq, dk, dv
+    torch.cuda.empty_cache()
+    return {"ms": ms, "steps": steps, "window": (t_host0, t_host1), "status": status}
+
+
 def cpu_baseline(w, seconds: float):
     """The float64 oracle's recurrence on a bounded prefix of the workload:
     batch row 0, all H heads, the first n tokens (n sized to ~`seconds`)."""
@@ -374,6 +415,7 @@ def main_ours(args):
     pre = bench_prefill(args, dist, w, dev)
     sampler.mark(*pre["window"])
     dec = None if args.no_decode else bench_decode(args, dist, dev)
+    bwd = None if args.backward_steps <= 0 else bench_backward(args, dist, w, dev)
     clocks = sampler.stop()
     tokens_step = w.B * w.N
     ms_step = pre["total_ms"] / args.steps
@@ -421,6 +463,21 @@ def main_ours(args):
                           "gpu_launches": dec["steps"], "state_finite": dec["finite"],
                           "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                                        "frac": gbs / hbm, "bytes_per_launch": dec["bytes"]}}
+    if bwd:
+        # minimal traffic of the operation: q, k, v, dout read once (bf16), dq,
+        # dk, dv written once (fp32); the three launches move 3 x 1280 B instead
+        units = w.B * w.H * w.N
+        bytes_min = units * (2 * (2 * w.D + 2 * w.E) + 4 * (2 * w.D + w.E))
+        bytes_moved = units * (3 * (2 * (w.D + w.D + w.E)) + 4 * (2 * w.D + w.E)) if w.D == w.E \
+            else None
+        gbs = bytes_min / (bwd["ms"] / 1e3) / 1e9
+        line["backward"] = {"value": job_throughput(dist.world, tokens_step, bwd["ms"]),
+                            "unit": "tokens/s", "ms_per_step": bwd["ms"], "steps": bwd["steps"],
+                            "gpu_launches": 3 * bwd["steps"], "device_status": bwd["status"],
+                            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
+                                         "unit": "GB/s", "frac": gbs / hbm,
+                                         "bytes_per_step": bytes_min,
+                                         "bytes_moved_by_three_launches": bytes_moved}}
     if dist.rank == 0 and dist.world == 1 and args.cpu_seconds > 0:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if dist.rank == 0:
