@@ -73,10 +73,13 @@ def _load():
                                                       I64, I64, I]
             lib.la_oracle_backward_recurrent.argtypes = [P, P, P, P, I, P, P, P, P, I64, I64, I64,
                                                          I64, I64, I]
+            lib.la_oracle_fused_layer.argtypes = [P, P, P, P, I, P, P, ctypes.c_double, P, I64,
+                                                  I64, I64, I64, I64, I]
             for f in ("la_oracle_masked", "la_oracle_recurrent", "la_oracle_recurrent_sampled",
                       "la_oracle_blocked", "la_oracle_decode_step", "la_oracle_max_threads",
                       "la_oracle_masked_anticausal", "la_oracle_recurrent_anticausal",
-                      "la_oracle_backward_masked", "la_oracle_backward_recurrent"):
+                      "la_oracle_backward_masked", "la_oracle_backward_recurrent",
+                      "la_oracle_fused_layer"):
                 getattr(lib, f).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -225,6 +228,30 @@ def backward(q, k, v, dout, slopes, form: str = "recurrent", threads: int = 0):
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), dt, _ptr(s), _ptr(dq), _ptr(dk), _ptr(dv),
               B, H, N, D, E, threads), f"la_oracle_backward_{form}")
     return dq, dk, dv
+
+
+def fused_layer(q, k, v, gate, slopes, norm_weight, eps: float, threads: int = 0) -> np.ndarray:
+    """The layer around the operator, float64 [B,H,N,E]:
+    y = w * RMSNorm_E(o) * sigmoid(gate) with o the recurrence on (silu(q),
+    silu(k), silu(v)); the RMSNorm runs over each head's E outputs and w is
+    per channel, norm_weight [H, E] (or [H * E])."""
+    q, k, v, dt = _inputs(q, k, v)
+    g = np.ascontiguousarray(gate)
+    if g.dtype != q.dtype:
+        raise TypeError("gate must have the dtype of q, k, v")
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    if g.shape != (B, H, N, E):
+        raise ValueError("gate must be [B,H,N,E]")
+    w = np.ascontiguousarray(np.asarray(norm_weight, dtype=np.float32).reshape(-1))
+    if w.shape[0] != H * E:
+        raise ValueError("norm_weight must have H * E entries")
+    s = _slopes(slopes, H)
+    out = np.empty((B, H, N, E), dtype=np.float64)
+    _check(_load().la_oracle_fused_layer(_ptr(q), _ptr(k), _ptr(v), _ptr(g), dt, _ptr(s),
+                                         _ptr(w), float(eps), _ptr(out), B, H, N, D, E, threads),
+           "la_oracle_fused_layer")
+    return out
 
 
 def max_threads() -> int:

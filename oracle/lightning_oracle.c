@@ -43,6 +43,15 @@
  *          dv_s = sum_{t >= s} g^(t-s) (q_t . k_s) dout_t      (g = gamma)
  *        (the derivative of the masked sum written out term by term, and the
  *        same sums as recurrences: forward for dq, backward in time for dk, dv).
+ *
+ * The layer around the operator ("MiniMax-M1" model entry, linear-layer field:
+ * SiLU on Q, K, V; RMSNorm on the output; sigmoid gate on the output after the
+ * RMSNorm, before the output projection):
+ *   la_oracle_fused_layer
+ *        y_t = w * RMSNorm(o_t) * sigmoid(g_t), o = the recurrence on
+ *        (silu(q), silu(k), silu(v)), RMSNorm over each head's E outputs:
+ *        RMSNorm(o_t) = o_t / sqrt(mean_e(o_te^2) + eps); w per channel
+ *        (h * E + e); silu(x) = x / (1 + exp(-x)); sigmoid(x) = 1/(1+exp(-x)).
  */
 #include <math.h>
 #include <stdint.h>
@@ -499,6 +508,60 @@ int la_oracle_backward_recurrent(const void* q, const void* k, const void* v, co
     free(kt);
     free(vt);
     free(gt);
+  }
+  return 0;
+}
+
+static double silu(double x) { return x / (1.0 + exp(-x)); }
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+int la_oracle_fused_layer(const void* q, const void* k, const void* v, const void* gate, int dtype,
+                          const float* slopes, const float* norm_w, double eps, double* out,
+                          int64_t B, int64_t H, int64_t N, int64_t D, int64_t E, int nthreads) {
+  int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
+  if (rc) return rc;
+  if (!gate || !norm_w || !(eps >= 0.0)) return 1;
+  set_threads(nthreads);
+  int64_t BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    int64_t h = bh % H;
+    double gamma = exp(-(double)slopes[h]);
+    double* S = (double*)calloc((size_t)(D * E), sizeof(double));
+    double* qt = (double*)malloc(sizeof(double) * (size_t)D);
+    double* kt = (double*)malloc(sizeof(double) * (size_t)D);
+    double* vt = (double*)malloc(sizeof(double) * (size_t)E);
+    double* ot = (double*)malloc(sizeof(double) * (size_t)E);
+    double* Y = out + bh * N * E;
+    for (int64_t t = 0; t < N; ++t) {
+      in_row(qt, q, (bh * N + t) * D, D, dtype);
+      in_row(kt, k, (bh * N + t) * D, D, dtype);
+      in_row(vt, v, (bh * N + t) * E, E, dtype);
+      for (int64_t d = 0; d < D; ++d) {
+        qt[d] = silu(qt[d]);
+        kt[d] = silu(kt[d]);
+      }
+      for (int64_t e = 0; e < E; ++e) vt[e] = silu(vt[e]);
+      for (int64_t d = 0; d < D; ++d)
+        for (int64_t e = 0; e < E; ++e) S[d * E + e] = gamma * S[d * E + e] + kt[d] * vt[e];
+      double ms = 0.0;
+      for (int64_t e = 0; e < E; ++e) {
+        double acc = 0.0;
+        for (int64_t d = 0; d < D; ++d) acc += qt[d] * S[d * E + e];
+        ot[e] = acc;
+        ms += acc * acc;
+      }
+      double rinv = 1.0 / sqrt(ms / (double)E + eps);
+      for (int64_t e = 0; e < E; ++e) {
+        double g = in_at(gate, (bh * N + t) * E + e, dtype);
+        Y[t * E + e] = (double)norm_w[h * E + e] * ot[e] * rinv * sigmoid(g);
+      }
+    }
+    free(S);
+    free(qt);
+    free(kt);
+    free(vt);
+    free(ot);
   }
   return 0;
 }
