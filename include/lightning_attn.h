@@ -208,6 +208,29 @@ int lightning_attn_bwd(const void* q, const void* k, const void* v, const void* 
                        int D, int E, void* stream);
 
 /*
+ * The layer around the operator, fused into the prefill kernel ("MiniMax-M1"
+ * model entry, linear-layer field: SiLU on Q, K, V, RMSNorm on the output;
+ * gate field: a sigmoid gate on the output after the RMSNorm, before the
+ * output projection):
+ *   y_t = w_h * RMSNorm(o_t) * sigmoid(gate_t),   o = operator(silu(q), silu(k), silu(v))
+ *   RMSNorm(o_t) = o_t / sqrt(mean_e(o_te^2) + eps), over each head's E outputs
+ * (the pages do not say which axis the RMSNorm covers; this reading is the one
+ * a per-head store can compute).
+ *   q, k : bf16 [B][H][N][D], the raw projections (SiLU is applied here)
+ *   v    : bf16 [B][H][N][E], raw;   gate: bf16 [B][H][N][E], before the sigmoid
+ *   norm_weight: fp32 [H][E]   eps: finite, >= 0 (else LA_ERR_SHAPE)
+ *   out  : bf16 [B][H][N][E]
+ * SiLU is applied in shared memory as the tiles arrive (the MUFU tanh gives the
+ * sigmoids), the norm, weight and gate in the epilogue, which stores bf16:
+ * 256 B of output per token-head instead of 512.  Zero initial state; D, E in
+ * {64, 128}; contiguous tensors, 16-byte aligned (else LA_ERR_ALIGN); errors
+ * otherwise as lightning_attn_fwd.
+ */
+int lightning_attn_fwd_fused(const void* q, const void* k, const void* v, const void* gate,
+                             const float* slopes, const float* norm_weight, float eps, void* out,
+                             int B, int H, int N, int D, int E, void* stream);
+
+/*
  * Fault-injection hook for testing the bounded device-side waits (an interface
  * for tests; the pages have no counterpart).  Runs the chunked bf16 prefill
  * (D = E = 128, chunk a multiple of 128 with N > chunk) but hands out work

@@ -94,7 +94,8 @@ enum BarId : int {
   B_P1F = 32,  // phase 1: K/V pair loaded, one per pair slot (3)
   B_P1E = 35,  // phase 1: pair slot free again (3)
   B_KT = 38,   // phase 1: decayed K tile of a pair slot ready (3)
-  B_COUNT = 41
+  B_ACT = 41,  // fused layer: Q and K tiles of a block activated (2)
+  B_COUNT = 43
 };
 
 // Optional event trace (compiled only with -DLA_TRACE): %globaltimer stamps of
@@ -157,6 +158,36 @@ __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t x, float f) {
 // Multiplies the 64 bf16 of one 128-byte swizzled row by f, in place.  All 8
 // loads are issued before any store; the physical chunk order (c ^ row) keeps
 // 8 consecutive rows on distinct banks.
+// SiLU, x sigmoid(x), with sigmoid(x) = (1 + tanh(x / 2)) / 2 from the
+// hardware tanh (tanh.approx.f32, one MUFU operation per element).
+__device__ __forceinline__ float tanh_hw(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float sigmoid_hw(float x) { return fmaf(0.5f, tanh_hw(0.5f * x), 0.5f); }
+__device__ __forceinline__ float silu_hw(float x) { return x * sigmoid_hw(x); }
+__device__ __forceinline__ uint32_t silu_scale_bf16x2(uint32_t x, float f) {
+  return pack_bf16x2(f * silu_hw(bf16lo_to_f32(x)), f * silu_hw(bf16hi_to_f32(x)));
+}
+
+// f * SiLU of the 64 bf16 of one 128-byte swizzled row, in place (the fused
+// layer's activation of q, k and v as they arrive in shared memory).
+__device__ __forceinline__ void silu_row(uint32_t rowaddr, uint32_t row, float f) {
+  uint4 x[8];
+#pragma unroll
+  for (uint32_t c = 0; c < 8; ++c) x[c] = lds128(rowaddr + ((c ^ (row & 7u)) << 4));
+#pragma unroll
+  for (uint32_t c = 0; c < 8; ++c) {
+    x[c].x = silu_scale_bf16x2(x[c].x, f);
+    x[c].y = silu_scale_bf16x2(x[c].y, f);
+    x[c].z = silu_scale_bf16x2(x[c].z, f);
+    x[c].w = silu_scale_bf16x2(x[c].w, f);
+  }
+#pragma unroll
+  for (uint32_t c = 0; c < 8; ++c) sts128(rowaddr + ((c ^ (row & 7u)) << 4), x[c]);
+}
+
 __device__ __forceinline__ void scale_row(uint32_t rowaddr, uint32_t row, float f) {
   uint4 x[8];
 #pragma unroll
@@ -413,6 +444,7 @@ __device__ void producer(const Ctx& c, const Params& p, const CUtensorMap* tq,
 // ---------------------------------------------------------------------------
 // MMA issuer: one thread issues every tcgen05.mma.
 // ---------------------------------------------------------------------------
+template <bool FUSED>
 __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
   constexpr uint32_t ID_KMAJ = idesc_bf16_f32(128, 128, false, false);  // Q K^T
   constexpr uint32_t ID_BMN = idesc_bf16_f32(128, 128, false, true);    // Q~ S, P V
@@ -427,6 +459,8 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
     const uint32_t qs = qi & 1u, ks = ki & 1u, buf = gidx & 1u;
     if (!wait_bar(c, p, B_QF + qs, (qi >> 1) & 1u)) return false;
     if (!wait_bar(c, p, B_KF + ks, (ki >> 1) & 1u)) return false;
+    // fused layer: group X activates (SiLU) Q and K in place first
+    if (FUSED && !wait_bar(c, p, B_ACT + buf, (gidx >> 1) & 1u)) return false;
     if (gidx >= 2 && !wait_bar(c, p, B_SE + buf, ((gidx >> 1) - 1) & 1u)) return false;
     LA_TRACE_EVENT(4, gidx);
     tc_fence_after();
@@ -519,8 +553,9 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
 
 // Runs the issue loop, then waits (bounded) until every MMA it issued has
 // completed, so TMEM is never released under a running MMA.
+template <bool FUSED>
 __device__ void mma_issuer(const Ctx& c, const Params& p) {
-  mma_issue_loop(c, p);
+  mma_issue_loop<FUSED>(c, p);
   mma_commit(&c.bar[B_DRAIN]);
   mbar_wait(&c.bar[B_DRAIN], 0, p.wait_limit_ns);
 }
@@ -528,7 +563,7 @@ __device__ void mma_issuer(const Ctx& c, const Params& p) {
 // ---------------------------------------------------------------------------
 // Group X: decay-causal mask and the in-place operand decays.
 // ---------------------------------------------------------------------------
-template <bool REV>
+template <bool REV, bool FUSED>
 __device__ void group_x(const Ctx& c, const Params& p) {
   const uint32_t t = threadIdx.x - 32u * X_WARP0;  // 0..255
   const uint32_t warp = t >> 5;
@@ -537,6 +572,18 @@ __device__ void group_x(const Ctx& c, const Params& p) {
   const uint32_t lane_base = ((warp & 3u) * 32u) << 16;
   const uint32_t gtab = c.sbase + OFF_GTAB;
   uint32_t q_it = 0, k_it = 0, w_it = 0, gb = 0, xs_n = 0, p1_it = 0;
+  // fused layer: SiLU on the Q and K tiles of phase-2 block gidx in place, then
+  // the MMA issuer may compute their scores
+  auto activate_qk = [&](uint32_t qi, uint32_t ki, uint32_t gidx) -> bool {
+    if (!cwait(c, p, B_QF + (qi & 1u), (qi >> 1) & 1u) ||
+        !cwait(c, p, B_KF + (ki & 1u), (ki >> 1) & 1u))
+      return false;
+    silu_row(c.sbase + OFF_Q + (qi & 1u) * TILE + hf * PLANE + r * 128u, r, 1.f);
+    silu_row(c.sbase + OFF_K + (ki & 1u) * TILE + hf * PLANE + r * 128u, r, 1.f);
+    fence_proxy_async_smem();
+    warp_arrive(&c.bar[B_ACT + (gidx & 1u)]);
+    return true;
+  };
   for (;;) {
     const uint32_t ws = w_it & 1u;
     if (!cwait(c, p, B_WF + ws, (w_it >> 1) & 1u)) break;
@@ -560,13 +607,19 @@ __device__ void group_x(const Ctx& c, const Params& p) {
         // reversed chunk-local index of this tile row (REV: row r is 127 - r)
         const int jc = b * BLK + static_cast<int>(REV ? 127u - r : r);
         const float f = jc < it.Lc ? expf(-lam * static_cast<float>(it.Lc - 1 - jc)) : 0.f;
-        scale_row(c.sbase + p1_base(slot) + hf * PLANE + r * 128u, r, f);
+        if (FUSED) {  // SiLU on k (with its decay) and on v
+          silu_row(c.sbase + p1_base(slot) + hf * PLANE + r * 128u, r, f);
+          silu_row(c.sbase + p1_base(slot) + TILE + hf * PLANE + r * 128u, r, 1.f);
+        } else {
+          scale_row(c.sbase + p1_base(slot) + hf * PLANE + r * 128u, r, f);
+        }
         fence_proxy_async_smem();
         warp_arrive(&c.bar[B_KT + slot]);
         if (t == 0) LA_TRACE_EVENT(22, p1_it);
         ++p1_it;
       }
     }
+    if (FUSED && it.p2 && it.nb > 0 && ok) ok = activate_qk(q_it, k_it, gb);
     for (int n = 0; n < (it.p2 ? it.nb : 0) && ok; ++n) {
       const uint32_t g = gb;
       const int len = min(BLK, it.Lc - n * BLK);
@@ -611,6 +664,10 @@ __device__ void group_x(const Ctx& c, const Params& p) {
         }
       }
       tmem_st32(t_s, pk);
+      if (FUSED) {  // SiLU on V in place before the state and PV products read it
+        if (!cwait(c, p, B_VF + qs, (q_it >> 1) & 1u)) { ok = false; break; }
+        silu_row(c.sbase + OFF_V + qs * TILE + hf * PLANE + r * 128u, r, 1.f);
+      }
       // gamma^(r+1) Q (bf16) into the S buffer's free columns; the Q tile is then dead
       {
         // gamma^(i+1) for the (reversed, if REV) local index i of row r
@@ -641,6 +698,7 @@ __device__ void group_x(const Ctx& c, const Params& p) {
       ++q_it;
       ++k_it;
       ++gb;
+      if (FUSED && n + 1 < it.nb && !activate_qk(q_it, k_it, gb)) { ok = false; break; }
     }
     if (!ok) break;
   }
@@ -696,7 +754,7 @@ __device__ __forceinline__ void st_scan32(float* base, uint32_t r, uint32_t hf, 
                        __uint_as_float(x[4 * i + 2]), __uint_as_float(x[4 * i + 3])));
 }
 
-template <int RANK, bool REV>
+template <int RANK, bool REV, bool FUSED>
 __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
   const uint32_t t = threadIdx.x - 32u * Y_WARP0;  // 0..127
   const uint32_t r = t;                            // TMEM lane / tile row
@@ -911,6 +969,76 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         ++gb;
         continue;
       }
+      if (FUSED) {
+        // Fused layer: y = w * o / sqrt(mean_e(o^2) + eps) * sigmoid(gate) in
+        // bf16, staged in this block's V slot (128 rows x 128 bf16 = one tile,
+        // laid out like the input tiles) and written by one pair of TMA stores.
+        float ss = 0.f;
+#pragma unroll 1
+        for (uint32_t qq = 0; qq < 4; ++qq) {
+          uint32_t o[32];
+          tmem_ld32(t_o + 32u * qq, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            ss = fmaf(__uint_as_float(o[i]), __uint_as_float(o[i]), ss);
+        }
+        const float rinv = rsqrtf(ss / static_cast<float>(p.E) + p.eps);
+        const int tok = row + static_cast<int>(r);
+        const uint16_t* grow =
+            tok < p.N ? p.gate + (static_cast<int64_t>(it.seq) * p.N + tok) * p.E : nullptr;
+        const float* wrow = p.norm_w + static_cast<int64_t>(it.seq % p.H) * p.E;
+#pragma unroll 1
+        for (uint32_t qq = 0; qq < 4; ++qq) {
+          uint32_t o[32];
+          tmem_ld32(t_o + 32u * qq, o);
+          tmem_wait_ld();
+          if (qq == 3) {  // every TMEM read of O done
+            tc_fence_before();
+            warp_arrive(&c.bar[B_O_EMPTY]);
+          }
+#pragma unroll
+          for (uint32_t cc = 0; cc < 4; ++cc) {  // 8 columns at a time
+            const int col = 32 * static_cast<int>(qq) + 8 * static_cast<int>(cc);
+            uint4 gv = make_uint4(0u, 0u, 0u, 0u);
+            float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
+            if (col < p.E) {
+              if (grow) gv = __ldg(reinterpret_cast<const uint4*>(grow + col));
+              w0 = __ldg(reinterpret_cast<const float4*>(wrow + col));
+              w1 = __ldg(reinterpret_cast<const float4*>(wrow + col + 4));
+            }
+            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t yw[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float a = wv[2 * j] * rinv * __uint_as_float(o[8 * cc + 2 * j]) *
+                              sigmoid_hw(bf16lo_to_f32(gw[j]));
+              const float b = wv[2 * j + 1] * rinv * __uint_as_float(o[8 * cc + 2 * j + 1]) *
+                              sigmoid_hw(bf16hi_to_f32(gw[j]));
+              yw[j] = pack_bf16x2(a, b);
+            }
+            const uint32_t lc = (qq & 1u) * 4u + cc;  // 16-byte chunk within the 64-column plane
+            sts128(vtile + (qq >> 1) * PLANE + r * 128u + ((lc ^ (r & 7u)) << 4),
+                   make_uint4(yw[0], yw[1], yw[2], yw[3]));
+          }
+        }
+        fence_proxy_async_smem();
+        if (!gsync(c, p, B_YSYNC, ys_n)) { ok = false; break; }
+        if (leader) {
+          tile_store<RANK>(to, vtile_g, 0, row, it.seq, it.seq % p.H, it.seq / p.H, p.cslot[3],
+                           pol_out);
+          tile_store<RANK>(to, vtile_g + PLANE, 64, row, it.seq, it.seq % p.H, it.seq / p.H,
+                           p.cslot[3], pol_out);
+          bulk_commit_group();
+          bulk_wait_group_read<0>();
+          mbar_arrive(&c.bar[B_VE + vs]);
+        }
+        if (leader) LA_TRACE_EVENT(14, g);
+        ++v_it;
+        ++gb;
+        continue;
+      }
       uint32_t o0[32], o1[32];
       tmem_ld32(t_o, o0);
       tmem_ld32(t_o + 32u, o1);
@@ -963,7 +1091,9 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
 // leave up to 128 registers per thread.
 // RANK: 3 for contiguous head-major q, k, v, out; 4 for strided layouts.
 // REV: anti-causal (o_t sums s >= t), the same blocked form in reversed time.
-template <int RANK, bool REV>
+// FUSED: the layer around the operator (SiLU on q, k, v in shared memory;
+// per-head RMSNorm, weight and sigmoid gate on the output, stored as bf16).
+template <int RANK, bool REV, bool FUSED>
 __global__ void __launch_bounds__(THREADS, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
@@ -987,6 +1117,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&c.bar[B_VE + i], 1);
       mbar_init(&c.bar[B_SF + i], 1);
       mbar_init(&c.bar[B_SE + i], 1);
+      mbar_init(&c.bar[B_ACT + i], X_WARPS);
       mbar_init(&c.bar[B_WF + i], 1);
       mbar_init(&c.bar[B_WE + i], 1 + X_WARPS + Y_WARPS);
     }
@@ -1030,12 +1161,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == PRODUCER_WARP) {
     if (lane_id() == 0) producer<RANK, REV>(c, p, &tq, &tk, &tv);
   } else if (warp == MMA_WARP) {
-    if (lane_id() == 0) mma_issuer(c, p);
+    if (lane_id() == 0) mma_issuer<FUSED>(c, p);
     __syncwarp();
   } else if (warp < Y_WARP0) {
-    group_x<REV>(c, p);
+    group_x<REV, FUSED>(c, p);
   } else {
-    group_y<RANK, REV>(c, p, &to);
+    group_y<RANK, REV, FUSED>(c, p, &to);
   }
 
   tc_fence_before();

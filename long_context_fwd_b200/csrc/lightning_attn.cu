@@ -207,9 +207,9 @@ bool strides_ok(const Strides& st) {
 // The four tensor maps of the bf16 prefill: 3-D [B*H][N][cols] maps when
 // every tensor is contiguous head-major, else 4-D maps (p.cslot says where t,
 // h and b went).  *rank receives 3 or 4.
-bool build_maps(const void* q, const void* k, const void* v, const float* out, int B, int H, int N,
+bool build_maps(const void* q, const void* k, const void* v, const void* out, int B, int H, int N,
                 int D, int E, const Strides& st, CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv,
-                CUtensorMap* to, la::fwd::Params& p, int* rank) {
+                CUtensorMap* to, la::fwd::Params& p, int* rank, bool out_bf16 = false) {
   // Column extents D and E: a 64-wide tensor leaves the second 64-column half
   // of every 128-wide tile outside the map, so TMA fills it with zeros (no
   // memory traffic) and clips stores there; zero columns add nothing to any
@@ -229,9 +229,11 @@ bool build_maps(const void* q, const void* k, const void* v, const float* out, i
     return la::make_tmap_3d(tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, nseq, 64, 128) &&
            la::make_tmap_3d(tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, nseq, 64, 128) &&
            la::make_tmap_3d(tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, nseq, 64, 128) &&
-           la::make_tmap_3d(to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, E, N, nseq, 32, 128);
+           (out_bf16 ? la::make_tmap_3d(to, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, nseq, 64, 128)
+                     : la::make_tmap_3d(to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, E, N, nseq, 32, 128));
   }
   *rank = 4;
+  if (out_bf16) return false;  // the fused layer takes contiguous tensors only
   const uint64_t ext[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(H),
                            static_cast<uint64_t>(B)};
   CUtensorMap* maps[4] = {tq, tk, tv, to};
@@ -252,9 +254,11 @@ bool build_maps(const void* q, const void* k, const void* v, const float* out, i
 // attribute on every call: it belongs to the current device's context).
 int launch_fwd(int rank, bool rev, int grid, cudaStream_t stream, const CUtensorMap& tq,
                const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
-               const la::fwd::Params& p) {
-  auto kern = rank == 3 ? (rev ? la::fwd::fwd_bf16_kernel<3, true> : la::fwd::fwd_bf16_kernel<3, false>)
-                        : (rev ? la::fwd::fwd_bf16_kernel<4, true> : la::fwd::fwd_bf16_kernel<4, false>);
+               const la::fwd::Params& p, bool fused = false) {
+  using la::fwd::fwd_bf16_kernel;
+  auto kern = fused     ? fwd_bf16_kernel<3, false, true>
+              : rank == 3 ? (rev ? fwd_bf16_kernel<3, true, false> : fwd_bf16_kernel<3, false, false>)
+                          : (rev ? fwd_bf16_kernel<4, true, false> : fwd_bf16_kernel<4, false, false>);
   const cudaError_t attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::fwd::SMEM_BYTES);
   if (attr != cudaSuccess) return cuda_fail(attr);
@@ -262,12 +266,26 @@ int launch_fwd(int rank, bool rev, int grid, cudaStream_t stream, const CUtensor
   return launch_status();
 }
 
+// The fused layer's extra operands (lightning_attn_fwd_fused).
+struct FusedArgs {
+  const void* gate;
+  const float* norm_w;
+  float eps;
+};
+
 int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slopes,
-                  const float* init_state, float* final_state, float* out, int B, int H, int N,
+                  const float* init_state, float* final_state, void* out, int B, int H, int N,
                   int D, int E, int chunk, void* stream_ptr, const Strides* strides = nullptr,
                   bool reverse = false, int first_chunk = 0,
-                  unsigned long long wait_limit_ns = kWaitLimitNs) {
+                  unsigned long long wait_limit_ns = kWaitLimitNs,
+                  const FusedArgs* fused = nullptr) {
   if (!q || !k || !v || !slopes || !out) return LA_ERR_NULL;
+  if (fused) {
+    if (!fused->gate || !fused->norm_w) return LA_ERR_NULL;
+    if (!aligned16(fused->gate) || !aligned16(fused->norm_w)) return LA_ERR_ALIGN;
+    if (!(fused->eps >= 0.f) || fused->eps > 3.0e38f) return LA_ERR_SHAPE;
+    if (strides || reverse) return LA_ERR_UNSUPPORTED;
+  }
   if (!dims_ok(B, H, N, D, E)) return LA_ERR_SHAPE;
   if ((D != 64 && D != 128) || (E != 64 && E != 128)) return LA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(slopes) ||
@@ -285,9 +303,15 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   la::fwd::Params p{};
   CUtensorMap tq, tk, tv, to;
   int rank = 3;
-  if (!build_maps(q, k, v, out, B, H, N, D, E, st, &tq, &tk, &tv, &to, p, &rank))
+  if (!build_maps(q, k, v, out, B, H, N, D, E, st, &tq, &tk, &tv, &to, p, &rank,
+                  fused != nullptr))
     return LA_ERR_CUDA;
-  p.out = out;
+  p.out = fused ? nullptr : static_cast<float*>(out);
+  if (fused) {
+    p.gate = static_cast<const uint16_t*>(fused->gate);
+    p.norm_w = fused->norm_w;
+    p.eps = fused->eps;
+  }
   for (int j = 0; j < 3; ++j) p.ostride[j] = st.s[3][j];
 
   p.slopes = slopes;
@@ -313,7 +337,7 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
     set_scratch(pl, scratch, p);
   }
 
-  int rc = launch_fwd(rank, reverse, pl.grid, stream, tq, tk, tv, to, p);
+  int rc = launch_fwd(rank, reverse, pl.grid, stream, tq, tk, tv, to, p, fused != nullptr);
   if (scratch) {
     const cudaError_t e = cudaFreeAsync(scratch, stream);
     if (e != cudaSuccess && rc == LA_OK) rc = cuda_fail(e);
@@ -472,6 +496,14 @@ int lightning_attn_bwd(const void* q, const void* k, const void* v, const void* 
   // dv_s = sum_{t>=s} g^(t-s) (k_s . q_t) dout_t: the anti-causal operator on (k, q, dout)
   return fwd_bf16_impl(k, q, dout, slopes, nullptr, nullptr, dv, B, H, N, D, E, 0, stream, nullptr,
                        true);
+}
+
+int lightning_attn_fwd_fused(const void* q, const void* k, const void* v, const void* gate,
+                             const float* slopes, const float* norm_weight, float eps, void* out,
+                             int B, int H, int N, int D, int E, void* stream) {
+  const FusedArgs fa{gate, norm_weight, eps};
+  return fwd_bf16_impl(q, k, v, slopes, nullptr, nullptr, out, B, H, N, D, E, 0, stream, nullptr,
+                       false, 0, kWaitLimitNs, &fa);
 }
 
 int lightning_attn_fault_test_scan_stall(const void* q, const void* k, const void* v,

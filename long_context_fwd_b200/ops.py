@@ -37,6 +37,8 @@ SIGNATURES = {
     "lightning_attn_device_status": [_P, _I],
     "lightning_attn_fwd_plan": [_I, _I, _I, _I, _I, _P, _P, _I, _P],
     "lightning_attn_fwd_anticausal": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P],
+    "lightning_attn_fwd_fused": [_P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _I, _I, _I, _I, _I,
+                                 _P],
     "lightning_attn_bwd": [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P],
     "lightning_attn_fwd_strided": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P,
                                    _I, _P],
@@ -195,6 +197,28 @@ def fwd_anticausal(q, k, v, slopes, out=None, *, init_state=None, final_state=No
         None if final_state is None else final_state.data_ptr(),
         out.data_ptr(), B, H, N, D, E, int(chunk), _stream_handle(stream))
     _check("lightning_attn_fwd_anticausal", rc)
+    return out
+
+
+def fwd_fused(q, k, v, gate, slopes, norm_weight, eps: float = 1e-6, out=None, *,
+              stream=None) -> torch.Tensor:
+    """The fused layer: raw bf16 q, k [B,H,N,D], v, gate [B,H,N,E], fp32 norm_weight
+    [H,E] -> bf16 w * RMSNorm_E(attention(silu(q), silu(k), silu(v))) * sigmoid(gate)."""
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    _need(q, "q", torch.bfloat16, (B, H, N, D))
+    _need(k, "k", torch.bfloat16, (B, H, N, D))
+    _need(v, "v", torch.bfloat16, (B, H, N, E))
+    _need(gate, "gate", torch.bfloat16, (B, H, N, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    _need(norm_weight, "norm_weight", torch.float32, (H, E))
+    if out is None:
+        out = torch.empty((B, H, N, E), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, (B, H, N, E))
+    rc = lib().lightning_attn_fwd_fused(q.data_ptr(), k.data_ptr(), v.data_ptr(), gate.data_ptr(),
+                                        slopes.data_ptr(), norm_weight.data_ptr(), float(eps),
+                                        out.data_ptr(), B, H, N, D, E, _stream_handle(stream))
+    _check("lightning_attn_fwd_fused", rc)
     return out
 
 

@@ -138,3 +138,15 @@ def test_backward_and_anticausal_validation(lib):
     g = lib.lightning_attn_fwd_anticausal
     assert g(None, FAKE, FAKE, FAKE, None, None, FAKE, 1, 1, 8, 128, 128, 0, None) == LA_ERR_NULL
     assert g(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 1, 8, 128, 128, 100, None) == LA_ERR_SHAPE
+
+
+def test_fused_layer_validation(lib):
+    f = lib.lightning_attn_fwd_fused
+    ok = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert f(FAKE, FAKE, FAKE, None, FAKE, FAKE, 1e-6, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1e-6, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, FAKE + 8, FAKE, FAKE, 1e-6, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_ALIGN
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4, 1e-6, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_ALIGN
+    assert f(*ok[:6], -1.0, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_SHAPE
+    assert f(*ok[:6], float("nan"), FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_SHAPE
+    assert f(*ok[:6], 1e-6, FAKE, 1, 1, 8, 128, 96, None) == LA_ERR_UNSUPPORTED

@@ -1,0 +1,70 @@
+"""GPU parity of the fused layer (lightning_attn_fwd_fused) against the oracle.
+
+Raw bf16 q, k, v and gate go in; the kernel applies SiLU to q, k, v in shared
+memory, runs the operator, and stores bf16 w * RMSNorm_E(o) * sigmoid(gate).
+Compared element by element (bf16 output upcast) with the float64 oracle's
+fused layer (pinned in tests/test_oracle_layer.py) on the same inputs, across
+the kernel's work splits, ragged lengths, 64-wide heads and gate/eps extremes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_fwd_b200 import inputs as I
+from long_context_fwd_b200 import ops
+from parity import TOL_BF16, bf16_to_dev, f32_to_dev, rel, worst_head
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+def _case(B, H, N, D, E, seed, gate_scale=2.0):
+    """Raw projections ~ N(0, 1) (the layer applies SiLU itself), gate ~ N(0, gate_scale^2)."""
+    rng = np.random.default_rng(1000 + seed)
+    raw = [I.f32_to_bf16_bits(rng.standard_normal(s).astype(np.float32))
+           for s in ((B, H, N, D), (B, H, N, D), (B, H, N, E))]
+    gate = I.f32_to_bf16_bits((rng.standard_normal((B, H, N, E)) * gate_scale).astype(np.float32))
+    w = (1.0 + 0.25 * rng.standard_normal((H, E))).astype(np.float32)
+    sl = I.alibi_slopes(H)
+    sl[1::4] = 0.0
+    return raw, gate, w, sl
+
+
+def _run(raw, gate, w, sl, eps):
+    q, k, v = (bf16_to_dev(x, DEV) for x in raw)
+    out = ops.fwd_fused(q, k, v, bf16_to_dev(gate, DEV), f32_to_dev(sl, DEV),
+                        f32_to_dev(w, DEV), eps)
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0
+    return out.float().cpu().numpy()
+
+
+FUSED_CASES = [
+    # B, H, N, D, E: whole sequences, split scan, hand-over, chunk scan, ragged, 64-wide
+    (2, 3, 777, 128, 128),
+    (1, 64, 2500, 128, 128),
+    (2, 80, 600, 128, 128),
+    (1, 4, 20000, 128, 128),
+    (1, 2, 129, 128, 128),
+    (1, 3, 1000, 64, 128),
+    (1, 2, 700, 128, 64),
+]
+
+
+@pytest.mark.parametrize("B,H,N,D,E", FUSED_CASES)
+def test_fused_layer_parity(B, H, N, D, E):
+    raw, gate, w, sl = _case(B, H, N, D, E, seed=N % 53 + H)
+    got = _run(raw, gate, w, sl, 1e-6)
+    ref = oracle.fused_layer(*raw, gate, sl, w, 1e-6)
+    assert np.isfinite(got).all()
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("eps,gate_scale", [(0.0, 0.0), (1e-2, 8.0), (1.0, 2.0)])
+def test_fused_layer_eps_and_gate_ranges(eps, gate_scale):
+    raw, gate, w, sl = _case(1, 4, 1500, 128, 128, seed=7, gate_scale=gate_scale)
+    got = _run(raw, gate, w, sl, eps)
+    ref = oracle.fused_layer(*raw, gate, sl, w, eps)
+    assert rel(got, ref) <= TOL_BF16

@@ -8,7 +8,7 @@ the RMSNorm, before the output projection):
 
 checked against an independent pure-Python statement built on the brute force
 of the operator, against closed forms of SiLU, sigmoid and RMSNorm, and
-against invariances (scale invariance of RMSNorm, gate limits), so that a
+against invariances (per-head independence, weight homogeneity, gate limits), so that a
 missing activation, a norm over the wrong axis or a misplaced weight fails.
 """
 import math
