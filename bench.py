@@ -110,6 +110,8 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--backward-steps", type=int, default=20,
                     help="steps of the backward-pass leg (0 skips it)")
+    ap.add_argument("--fused-steps", type=int, default=20,
+                    help="steps of the fused-layer leg (0 skips it)")
     return ap.parse_args()
 
 
@@ -368,6 +370,44 @@ def bench_backward(args, dist, w, dev):
     return {"ms": ms, "steps": steps, "window": (t_host0, t_host1), "status": status}
 
 
+def bench_fused(args, dist, w, dev):
+    """The fused layer (SiLU on raw q, k, v; per-head RMSNorm, weight and sigmoid
+    gate on the output; bf16 out) on the prefill workload's shapes, inputs
+    resident on the device."""
+    import torch
+    from long_context_fwd_b200 import inputs as I
+    from long_context_fwd_b200 import ops
+
+    g = torch.Generator(device=dev)
+    g.manual_seed(24680)
+    q, k = (torch.randn((w.B, w.H, w.N, w.D), generator=g, device=dev).to(torch.bfloat16)
+            for _ in range(2))
+    v, gate = (torch.randn((w.B, w.H, w.N, w.E), generator=g, device=dev).to(torch.bfloat16)
+               for _ in range(2))
+    nw = torch.ones((w.H, w.E), dtype=torch.float32, device=dev)
+    sl = torch.from_numpy(I.slopes_for(w)).to(dev)
+    out = torch.empty((w.B, w.H, w.N, w.E), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        ops.fwd_fused(q, k, v, gate, sl, nw, 1e-6, out)
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0, "device-side wait timed out during warm-up"
+    dist.barrier()
+    steps = args.fused_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        ops.fwd_fused(q, k, v, gate, sl, nw, 1e-6, out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = dist.max(e0.elapsed_time(e1)) / steps
+    status = ops.device_status(reset=True)
+    del q, k, v, gate, out
+    torch.cuda.empty_cache()
+    return {"ms": ms, "steps": steps, "status": status}
+
+
 def cpu_baseline(w, seconds: float):
     """The float64 oracle's recurrence on a bounded prefix of the workload:
     batch row 0, all H heads, the first n tokens (n sized to ~`seconds`)."""
@@ -416,6 +456,7 @@ def main_ours(args):
     sampler.mark(*pre["window"])
     dec = None if args.no_decode else bench_decode(args, dist, dev)
     bwd = None if args.backward_steps <= 0 else bench_backward(args, dist, w, dev)
+    fus = None if args.fused_steps <= 0 else bench_fused(args, dist, w, dev)
     clocks = sampler.stop()
     tokens_step = w.B * w.N
     ms_step = pre["total_ms"] / args.steps
@@ -478,6 +519,18 @@ def main_ours(args):
                                          "unit": "GB/s", "frac": gbs / hbm,
                                          "bytes_per_step": bytes_min,
                                          "bytes_moved_by_three_launches": bytes_moved}}
+    if fus:
+        # the layer's traffic: raw q, k, v and the gate in (bf16), y out (bf16)
+        units = w.B * w.H * w.N
+        bytes_layer = units * 2 * (2 * w.D + 3 * w.E)
+        gbs = bytes_layer / (fus["ms"] / 1e3) / 1e9
+        line["fused_layer"] = {"value": job_throughput(dist.world, tokens_step, fus["ms"]),
+                               "unit": "tokens/s", "ms_per_step": fus["ms"],
+                               "steps": fus["steps"], "gpu_launches": fus["steps"],
+                               "device_status": fus["status"],
+                               "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
+                                            "unit": "GB/s", "frac": gbs / hbm,
+                                            "bytes_per_step": bytes_layer}}
     if dist.rank == 0 and dist.world == 1 and args.cpu_seconds > 0:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if dist.rank == 0:
