@@ -158,17 +158,22 @@ __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t x, float f) {
 // Multiplies the 64 bf16 of one 128-byte swizzled row by f, in place.  All 8
 // loads are issued before any store; the physical chunk order (c ^ row) keeps
 // 8 consecutive rows on distinct banks.
-// SiLU, x sigmoid(x), with sigmoid(x) = (1 + tanh(x / 2)) / 2 from the
-// hardware tanh (tanh.approx.f32, one MUFU operation per element).
+// sigmoid(x) = (1 + tanh(x / 2)) / 2 from the hardware tanh (tanh.approx.f32,
+// one MUFU operation per element): the fused layer's gate.
 __device__ __forceinline__ float tanh_hw(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 __device__ __forceinline__ float sigmoid_hw(float x) { return fmaf(0.5f, tanh_hw(0.5f * x), 0.5f); }
-__device__ __forceinline__ float silu_hw(float x) { return x * sigmoid_hw(x); }
+
+// f * SiLU of a bf16 pair, f x sigmoid(x), in fp32 and rounded once (one MUFU
+// operation per element).  Packed bf16 arithmetic with the bf16 tanh was
+// tried: its error reached 7% on heads with fast decay, where few tokens
+// average it out, so it is not used.
 __device__ __forceinline__ uint32_t silu_scale_bf16x2(uint32_t x, float f) {
-  return pack_bf16x2(f * silu_hw(bf16lo_to_f32(x)), f * silu_hw(bf16hi_to_f32(x)));
+  const float lo = bf16lo_to_f32(x), hi = bf16hi_to_f32(x);
+  return pack_bf16x2(f * lo * sigmoid_hw(lo), f * hi * sigmoid_hw(hi));
 }
 
 // f * SiLU of the 64 bf16 of one 128-byte swizzled row, in place (the fused
@@ -973,6 +978,19 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         // Fused layer: y = w * o / sqrt(mean_e(o^2) + eps) * sigmoid(gate) in
         // bf16, staged in this block's V slot (128 rows x 128 bf16 = one tile,
         // laid out like the input tiles) and written by one pair of TMA stores.
+        // The row's gate is first copied (cp.async) into exactly the positions
+        // its outputs will take, while the row's mean square is computed; each
+        // output chunk then overwrites its own gate chunk.
+        const int tok = row + static_cast<int>(r);
+        const uint16_t* grow =
+            tok < p.N ? p.gate + (static_cast<int64_t>(it.seq) * p.N + tok) * p.E : nullptr;
+        const uint32_t srow = vtile + r * 128u;
+        if (grow) {
+#pragma unroll
+          for (uint32_t ch = 0; ch < 16; ++ch)  // 16-byte chunk ch: plane ch / 8, chunk ch % 8
+            if (static_cast<int>(8 * ch) < p.E)
+              cp_async16(srow + (ch >> 3) * PLANE + (((ch & 7u) ^ (r & 7u)) << 4), grow + 8 * ch);
+        }
         float ss = 0.f;
 #pragma unroll 1
         for (uint32_t qq = 0; qq < 4; ++qq) {
@@ -984,10 +1002,8 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
             ss = fmaf(__uint_as_float(o[i]), __uint_as_float(o[i]), ss);
         }
         const float rinv = rsqrtf(ss / static_cast<float>(p.E) + p.eps);
-        const int tok = row + static_cast<int>(r);
-        const uint16_t* grow =
-            tok < p.N ? p.gate + (static_cast<int64_t>(it.seq) * p.N + tok) * p.E : nullptr;
         const float* wrow = p.norm_w + static_cast<int64_t>(it.seq % p.H) * p.E;
+        cp_async_wait_all();
 #pragma unroll 1
         for (uint32_t qq = 0; qq < 4; ++qq) {
           uint32_t o[32];
@@ -1000,12 +1016,14 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
 #pragma unroll
           for (uint32_t cc = 0; cc < 4; ++cc) {  // 8 columns at a time
             const int col = 32 * static_cast<int>(qq) + 8 * static_cast<int>(cc);
-            uint4 gv = make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t lc = (qq & 1u) * 4u + cc;  // 16-byte chunk within the 64-column plane
+            const uint32_t addr = srow + (qq >> 1) * PLANE + ((lc ^ (r & 7u)) << 4);
             float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
+            uint4 gv = make_uint4(0u, 0u, 0u, 0u);
             if (col < p.E) {
-              if (grow) gv = __ldg(reinterpret_cast<const uint4*>(grow + col));
               w0 = __ldg(reinterpret_cast<const float4*>(wrow + col));
               w1 = __ldg(reinterpret_cast<const float4*>(wrow + col + 4));
+              if (grow) gv = lds128(addr);
             }
             const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
             const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
@@ -1018,9 +1036,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
                               sigmoid_hw(bf16hi_to_f32(gw[j]));
               yw[j] = pack_bf16x2(a, b);
             }
-            const uint32_t lc = (qq & 1u) * 4u + cc;  // 16-byte chunk within the 64-column plane
-            sts128(vtile + (qq >> 1) * PLANE + r * 128u + ((lc ^ (r & 7u)) << 4),
-                   make_uint4(yw[0], yw[1], yw[2], yw[3]));
+            sts128(addr, make_uint4(yw[0], yw[1], yw[2], yw[3]));
           }
         }
         fence_proxy_async_smem();
