@@ -73,8 +73,15 @@ constexpr uint32_t OFF_KVB = 6 * TILE;  // bf16 copy of the state (MMA B operand
 constexpr uint32_t OFF_BAR = 7 * TILE;
 constexpr uint32_t OFF_GTAB = OFF_BAR + 512;  // 256 floats: gtab[u] = gamma^(127-u), 0 for u > 127
 constexpr uint32_t OFF_MISC = OFF_GTAB + 1024;
-constexpr uint32_t SMEM_USED = OFF_MISC + 128;
+// split scan: the pieces an entering state chains, (slot, blocks from the
+// piece's end to the share's start) pairs written by group Y's leader.  The
+// host takes the split only for at least SMs/8 sequences, so a chain holds
+// at most G/nseq + G2/nseq + 3 <= 19 pieces.
+constexpr int CHAIN_MAX = 32;
+constexpr uint32_t OFF_CHAIN = OFF_MISC + 128;
+constexpr uint32_t SMEM_USED = OFF_CHAIN + 8 * CHAIN_MAX;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 227u * 1024u, "dynamic shared memory above the per-CTA limit");
 
 constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_KV = 384;
 
@@ -248,7 +255,9 @@ struct Ctx {
   uint32_t sbase;           // shared-space address of sm
   uint64_t* bar;
   volatile uint32_t* misc;  // [0] TMEM base, [1..2] work slots, [3] abort,
-                            // [4..17] this CTA's share of a static split
+                            // [4..17] this CTA's share of a static split,
+                            // [18] length of the chain below
+  volatile uint32_t* chain;  // CHAIN_MAX (slot, distance) pairs
   uint32_t tmem;
 };
 
@@ -801,14 +810,24 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     const int64_t x_hi = x_lo + it.t0 / BLK;
     if (it.enter) {
       if (leader) {
+        // wait for each piece in turn and note it in the chain list
         const uint64_t t0 = globaltimer_ns();
         uint32_t spins = 0;
         int64_t x = x_lo;
         int slot = chain ? s1_slot(p, G, x) : it.enter_slot;
+        uint32_t n = 0;
         for (;;) {
           if (ld_acquire_gpu(p.flags + slot) == it.enter_val) {
             if (!chain) break;
-            x = s1_next(p, G, x);
+            const int64_t y = s1_next(p, G, x);
+            if (n == CHAIN_MAX) {  // excluded by the host's plan; no wrong result
+              fail(c, p, 4);
+              break;
+            }
+            c.chain[2 * n] = static_cast<uint32_t>(slot);
+            c.chain[2 * n + 1] = static_cast<uint32_t>(x_hi - y);
+            ++n;
+            x = y;
             if (x >= x_hi) break;
             slot = s1_slot(p, G, x);
             continue;
@@ -818,6 +837,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
             break;
           }
         }
+        c.misc[18] = n;
       }
       if (!gsync(c, p, B_YSYNC, ys_n)) break;
       if (!chain) scan_src = p.prefix + static_cast<int64_t>(it.enter_slot) * (HD * HD);
@@ -846,17 +866,19 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
           for (int i = 0; i < 32; ++i) prev[i] = 0u;
         }
         if (chain) {
+          // S(X) = gamma^(128 (X - x_lo)) S(x_lo) + sum_j gamma^(128 (X - y_j)) piece_j
+          const int n = static_cast<int>(c.misc[18]);
+          const float g_all = expf(-lam * static_cast<float>((x_hi - x_lo) * BLK));
+#pragma unroll
+          for (int i = 0; i < 32; ++i) prev[i] = __float_as_uint(g_all * __uint_as_float(prev[i]));
 #pragma unroll 1
-          for (int64_t x = x_lo; x < x_hi;) {
-            const int64_t y = s1_next(p, G, x);
-            const float gp = expf(-lam * static_cast<float>((y - x) * BLK));
+          for (int j = 0; j < n; ++j) {
             uint32_t part[32];
-            ld_scan32(p.prefix + static_cast<int64_t>(s1_slot(p, G, x)) * (HD * HD), r, q >> 1, q & 1u,
-                      part);
+            ld_scan32(p.prefix + static_cast<int64_t>(c.chain[2 * j]) * (HD * HD), r, q >> 1, q & 1u, part);
+            const float w = expf(-lam * static_cast<float>(static_cast<int>(c.chain[2 * j + 1]) * BLK));
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              prev[i] = __float_as_uint(fmaf(gp, __uint_as_float(prev[i]), __uint_as_float(part[i])));
-            x = y;
+              prev[i] = __float_as_uint(fmaf(w, __uint_as_float(part[i]), __uint_as_float(prev[i])));
           }
         }
         if (it.phase1) {
@@ -1121,6 +1143,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   c.sbase = smem_u32(c.sm);
   c.bar = reinterpret_cast<uint64_t*>(c.sm + OFF_BAR);
   c.misc = reinterpret_cast<volatile uint32_t*>(c.sm + OFF_MISC);
+  c.chain = reinterpret_cast<volatile uint32_t*>(c.sm + OFF_CHAIN);
   const uint32_t warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {

@@ -181,6 +181,8 @@ def test_split_scan(B, H, N, sms):
                     assert local[x][0] == ln["b"] and local[x][2] == ln["enter_slot"]
                     x = ln["b"]
                 assert x == it["seq"] * F + it["a"] // BLK
+                # the kernel notes the chain in a 32-entry shared-memory list
+                assert len(links) <= 32
         kinds = [it["kind"] for it in its]
         # local-state items first, then outputs (the entering one last)
         first_out = kinds.index(0) if 0 in kinds else len(kinds)
