@@ -180,7 +180,9 @@ __device__ __forceinline__ float sigmoid_hw(float x) { return fmaf(0.5f, tanh_hw
 // average it out, so it is not used.
 __device__ __forceinline__ uint32_t silu_scale_bf16x2(uint32_t x, float f) {
   const float lo = bf16lo_to_f32(x), hi = bf16hi_to_f32(x);
-  return pack_bf16x2(f * lo * sigmoid_hw(lo), f * hi * sigmoid_hw(hi));
+  const float hl = 0.5f * lo, hh = 0.5f * hi;
+  const float fl = f * hl, fh = f * hh;
+  return pack_bf16x2(fmaf(fl, tanh_hw(hl), fl), fmaf(fh, tanh_hw(hh), fh));
 }
 
 // f * SiLU of the 64 bf16 of one 128-byte swizzled row, in place (the fused
@@ -522,8 +524,10 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
       const uint32_t ks = (k0 + n) & 1u, vs = (v0 + n) & 1u;
       if (!wait_bar(c, p, B_READY, ready_n++ & 1u)) return;
       LA_TRACE_EVENT(3, g);
-      // the next block's scores first, so group X can start on them
-      if (n + 1 < nb && !issue_S(q0 + n + 1, k0 + n + 1, g + 1)) return;
+      // the next block's scores first, so group X can start on them (the
+      // fused layer's scores wait for group X's activation of Q and K, so
+      // there they follow this block's products)
+      if (!FUSED && n + 1 < nb && !issue_S(q0 + n + 1, k0 + n + 1, g + 1)) return;
       if (!wait_bar(c, p, B_KVB_READY, kvb_n++ & 1u)) return;
       LA_TRACE_EVENT(5, g);
       if (!wait_bar(c, p, B_VF + vs, ((v0 + n) >> 1) & 1u)) return;
@@ -556,6 +560,7 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
       mma_commit(&c.bar[B_O_FULL]);
       mma_commit(&c.bar[B_SE + (g & 1u)]);
       LA_TRACE_EVENT(8, g);
+      if (FUSED && n + 1 < nb && !issue_S(q0 + n + 1, k0 + n + 1, g + 1)) return;
       // The V tile is released by group Y after it has staged the output there.
     }
     q_it += nb;
@@ -1025,7 +1030,9 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         }
         const float rinv = rsqrtf(ss / static_cast<float>(p.E) + p.eps);
         const float* wrow = p.norm_w + static_cast<int64_t>(it.seq % p.H) * p.E;
+        if (leader) LA_TRACE_EVENT(23, g);
         cp_async_wait_all();
+        if (leader) LA_TRACE_EVENT(24, g);
 #pragma unroll 1
         for (uint32_t qq = 0; qq < 4; ++qq) {
           uint32_t o[32];
@@ -1062,6 +1069,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
           }
         }
         fence_proxy_async_smem();
+        if (leader) LA_TRACE_EVENT(25, g);
         if (!gsync(c, p, B_YSYNC, ys_n)) { ok = false; break; }
         if (leader) {
           tile_store<RANK>(to, vtile_g, 0, row, it.seq, it.seq % p.H, it.seq / p.H, p.cslot[3],
@@ -1069,6 +1077,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
           tile_store<RANK>(to, vtile_g + PLANE, 64, row, it.seq, it.seq % p.H, it.seq / p.H,
                            p.cslot[3], pol_out);
           bulk_commit_group();
+          LA_TRACE_EVENT(26, g);
           bulk_wait_group_read<0>();
           mbar_arrive(&c.bar[B_VE + vs]);
         }
