@@ -524,10 +524,7 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
       const uint32_t ks = (k0 + n) & 1u, vs = (v0 + n) & 1u;
       if (!wait_bar(c, p, B_READY, ready_n++ & 1u)) return;
       LA_TRACE_EVENT(3, g);
-      // the next block's scores first, so group X can start on them (the
-      // fused layer's scores wait for group X's activation of Q and K, so
-      // there they follow this block's products)
-      if (!FUSED && n + 1 < nb && !issue_S(q0 + n + 1, k0 + n + 1, g + 1)) return;
+      // (the next block's scores follow this block's products)
       if (!wait_bar(c, p, B_KVB_READY, kvb_n++ & 1u)) return;
       LA_TRACE_EVENT(5, g);
       if (!wait_bar(c, p, B_VF + vs, ((v0 + n) >> 1) & 1u)) return;
@@ -560,7 +557,7 @@ __device__ void mma_issue_loop(const Ctx& c, const Params& p) {
       mma_commit(&c.bar[B_O_FULL]);
       mma_commit(&c.bar[B_SE + (g & 1u)]);
       LA_TRACE_EVENT(8, g);
-      if (FUSED && n + 1 < nb && !issue_S(q0 + n + 1, k0 + n + 1, g + 1)) return;
+      if (n + 1 < nb && !issue_S(q0 + n + 1, k0 + n + 1, g + 1)) return;
       // The V tile is released by group Y after it has staged the output there.
     }
     q_it += nb;
