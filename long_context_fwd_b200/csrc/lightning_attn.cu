@@ -400,9 +400,11 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
   la::fwd::Params p{};
   CUtensorMap tq, tk, tv, to;
   int rank = 3;
-  if (!build_maps(q, k, v, out, B, H, N, D, E, contiguous_strides(H, N, D, E), &tq, &tk, &tv, &to,
-                  p, &rank))
+  const Strides st = contiguous_strides(H, N, D, E);
+  if (!build_maps(q, k, v, out, B, H, N, D, E, st, &tq, &tk, &tv, &to, p, &rank))
     return LA_ERR_CUDA;
+  p.out = out;
+  for (int j = 0; j < 3; ++j) p.ostride[j] = st.s[3][j];
 
   p.slopes = slopes;
   p.status = status_word();
