@@ -287,6 +287,9 @@ const char* lightning_attn_status_string(int status);
  * Reads the calling thread's current device's sticky device-side status word
  * (LA_OK or LA_ERR_TIMEOUT) into *status; if reset != 0 clears it.  This call
  * synchronises with the device.  Returns LA_OK or LA_ERR_NULL / LA_ERR_CUDA.
+ * LA_ERR_TIMEOUT covers every device-side abort: a bounded wait that ran out,
+ * and (never expected: the host's work split excludes it) a split-scan share
+ * whose pieces would not fit the kernel's shared-memory lists.
  */
 int lightning_attn_device_status(int* status, int reset);
 

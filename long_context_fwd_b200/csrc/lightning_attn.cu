@@ -13,7 +13,8 @@
 
 namespace la {
 // Sticky device-side status word: bit 0 = an mbarrier wait ran out of time,
-// bit 1 = a chunk-scan flag wait ran out of time.
+// bit 1 = a chunk-scan flag wait ran out of time, bit 2 = a split-scan share
+// or chain exceeded its shared-memory list (excluded by the host's plan).
 __device__ int g_status;
 }  // namespace la
 
