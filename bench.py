@@ -51,36 +51,36 @@ def kernel_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(workload) -> "float | None":
+def measured_traffic(workload, sms: int) -> "float | None":
     """DRAM bytes per launch of the prefill kernel from the committed ncu summary,
     scaled to `workload` by (b, h, token) units; None unless the summary was
     taken on the current kernel source.  The summary holds one capture per way
     of splitting the work: whole sequences / the balanced hand-over
     (`dram_bytes_per_launch`) and the split scan (`split_dram_bytes_per_launch`,
     whose extra local-state reads scale with tokens only for the same number
-    of sequences, 64, as the 8K and 1M workloads)."""
+    of sequences, 64, as the 8K and 1M workloads).  `sms`: the device's SM
+    count, which decides the split."""
+    fields = {}
     try:
-        fields = {}
         with open(PROFILE) as f:
             for line in f:
                 if line.startswith("- ") and ":" in line:
                     k, v = line[2:].split(":", 1)
                     fields[k.strip()] = v.strip().strip("`")
-        if fields.get("kernel_sha") != kernel_hash():
-            return None
-        from long_context_fwd_b200 import ops
-        sms = torch.cuda.get_device_properties(0).multi_processor_count
-        mode = ops.fwd_plan(workload.B, workload.H, workload.N, 0, sms)[0]["mode"]
-        if mode == 2:
-            if workload.B * workload.H != int(fields["split_sequences"]):
-                return None
-            per_unit = (float(fields["split_dram_bytes_per_launch"]) /
-                        float(fields["split_token_heads_per_launch"]))
-        else:
-            per_unit = float(fields["dram_bytes_per_launch"]) / float(fields["token_heads_per_launch"])
-        return per_unit * workload.B * workload.H * workload.N
-    except Exception:
+    except OSError:
         return None
+    if fields.get("kernel_sha") != kernel_hash():
+        return None
+    from long_context_fwd_b200 import ops
+    mode = ops.fwd_plan(workload.B, workload.H, workload.N, 0, sms)[0]["mode"]
+    if mode == 2:
+        if workload.B * workload.H != int(fields["split_sequences"]):
+            return None
+        per_unit = (float(fields["split_dram_bytes_per_launch"]) /
+                    float(fields["split_token_heads_per_launch"]))
+    else:
+        per_unit = float(fields["dram_bytes_per_launch"]) / float(fields["token_heads_per_launch"])
+    return per_unit * workload.B * workload.H * workload.N
 
 
 def peaks():
@@ -270,14 +270,15 @@ def bench_prefill(args, dist, w, dev):
     dq, dk, dv = (torch.empty(x.shape, dtype=x.dtype, device=dev) for x in (hq, hk, hv))
 
     # The step runs as G groups of consecutive (b, h) sequences (whole batch rows,
-    # or equal runs of heads of one row) on two streams, so one group's inputs go
-    # up while another's result comes down (PCIe is full duplex): copy in,
-    # prefill, copy out per group.
+    # or equal runs of heads of one row): one stream copies every group's inputs
+    # up back to back, one runs each group's prefill once its inputs are in, one
+    # copies each group's result down once it is computed, so uploads run
+    # continuously and overlap the downloads (PCIe is full duplex).
     nseq = w.B * w.H
-    G = next((g for g in (8, 4, 2) if nseq % g == 0 and
+    G = next((g for g in (16, 8, 4, 2) if nseq % g == 0 and
               (w.H % (nseq // g) == 0 or (nseq // g) % w.H == 0)), 1)
     per = nseq // G
-    streams = [torch.cuda.Stream(device=dev) for _ in range(2)]
+    up, comp, down = (torch.cuda.Stream(device=dev) for _ in range(3))
 
     def group_views(i):
         lo = i * per
@@ -297,23 +298,28 @@ def bench_prefill(args, dist, w, dev):
             return
         start = torch.cuda.Event()
         start.record(stream)
-        done = []
-        for i in range(G):
-            st = streams[i % 2]
+        for st in (up, comp, down):
             st.wait_event(start)
+        for i in range(G):
             shp, hs = group_views(i)
-            with torch.cuda.stream(st):
-                gq, gk, gv, go = shp(dq), shp(dk), shp(dv), shp(out)
+            gq, gk, gv, go = shp(dq), shp(dk), shp(dv), shp(out)
+            with torch.cuda.stream(up):
                 gq.copy_(shp(hq), non_blocking=True)
                 gk.copy_(shp(hk), non_blocking=True)
                 gv.copy_(shp(hv), non_blocking=True)
-                ops.fwd(gq, gk, gv, sl[hs], go, chunk=args.chunk, stream=st)
+                landed = torch.cuda.Event()
+                landed.record(up)
+            comp.wait_event(landed)
+            with torch.cuda.stream(comp):
+                ops.fwd(gq, gk, gv, sl[hs], go, chunk=args.chunk, stream=comp)
+                computed = torch.cuda.Event()
+                computed.record(comp)
+            down.wait_event(computed)
+            with torch.cuda.stream(down):
                 shp(hout).copy_(go, non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(st)
-            done.append(ev)
-        for ev in done:
-            stream.wait_event(ev)
+        finished = torch.cuda.Event()
+        finished.record(down)
+        stream.wait_event(finished)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -509,6 +515,9 @@ def main_ours(args):
     bytes_launch = w.B * w.H * w.N * BYTES_PER_TOKEN_HEAD
     achieved = bytes_launch / (pre["launch_ms"] / 1e3) / 1e9
     flops_launch = w.B * w.H * w.N * (4 * w.D * w.E + 2 * BLK * (w.D + w.E))
+    # the committed capture is of head-major tensors
+    traffic = (measured_traffic(w, torch.cuda.get_device_properties(dev).multi_processor_count)
+               if args.layout == "head-major" else None)
     line = {
         "metric": METRIC,
         "value": value,
@@ -529,7 +538,7 @@ def main_ours(args):
                    "l2": f"no flush: each step streams {bytes_launch / 1e9:.2f} GB, larger than the "
                          "126 MB L2"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": measured_traffic(w),
+                     "frac": achieved / hbm, "traffic": traffic,
                      "peak_source": f"{peak_src} copy bandwidth",
                      "bytes_per_launch": bytes_launch, "kernel_ms": pre["launch_ms"],
                      "tensor_tflops": flops_launch / (pre["launch_ms"] / 1e3) / 1e12,
@@ -540,8 +549,8 @@ def main_ours(args):
             "value": job_throughput(dist.world, tokens_step, pre["e2e_ms"]), "unit": "tokens/s",
             "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"],
             "ms_per_step": pre["e2e_ms"],
-            "pipelining": f"{pre['e2e_groups']} groups of sequences on 2 streams "
-                          "(copy in, prefill, copy out per group)"},
+            "pipelining": f"{pre['e2e_groups']} groups of sequences: uploads, prefills and "
+                          "downloads on three streams, ordered per group by events"},
         "clocks": clocks,
     }
     if dec:
