@@ -89,7 +89,7 @@ def peaks():
         with open(path) as f:
             d = json.load(f)
         return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
-    except Exception:
+    except (OSError, KeyError, TypeError, ValueError):
         return 6650.0, 1590.0, "fallback"
 
 
@@ -170,7 +170,7 @@ class ClockSampler:
                 ["nvidia-smi", "-i", str(device_index), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.tmp, stderr=subprocess.DEVNULL)
-        except Exception:
+        except OSError:
             self.proc = None
         self.windows = []
 
@@ -183,7 +183,7 @@ class ClockSampler:
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
-        except Exception:
+        except subprocess.TimeoutExpired:
             self.proc.kill()
         self.tmp.flush()
         rows = []
@@ -196,7 +196,7 @@ class ClockSampler:
                     ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
                     ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
                     rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
-                except Exception:
+                except (ValueError, IndexError, OverflowError):
                     continue
         os.unlink(self.tmp.name)
         inside = [r for r in rows if any(a - 0.05 <= r[0] <= b + 0.05 for a, b in self.windows)]
