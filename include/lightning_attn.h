@@ -120,8 +120,9 @@ int lightning_attn_fwd_ex(const void* q, const void* k, const void* v,
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) and caches it; make that first call before any stream
  * capture.  All calls on a device share the one array and it keeps the last
- * call's contents (the counters are cleared with cudaMemsetAsync on `stream`
- * at every call): calls whose kernels overlap on the GPU -- e.g. issued on
+ * call's contents (the chunk scan's counters are cleared with cudaMemsetAsync
+ * on `stream` at every call; the other splits' flags carry a value unique to
+ * the call): calls whose kernels overlap on the GPU -- e.g. issued on
  * different streams without ordering between them -- race on it and must be
  * serialised by the caller.
  */
@@ -264,14 +265,17 @@ const char* lightning_attn_last_cuda_error(void);
  *   info[8]: mode (0 whole sequences / chunk scan with tickets, 1 balanced
  *            hand-over, 2 split scan), grid size, chunk length, chunks per
  *            sequence, split-scan first-part blocks F, split-scan output CTAs
- *            over the first parts G2, state slots, flag words.
+ *            over the first parts G2, state slots, 64-bit flags.
  *   rec[10 * i .. 10 * i + 9] for record i: cta (-1 for ticket items), kind
  *            (0 outputs, 1 local state only, 2 a local state chained into the
  *            preceding kind-0 record's entering state), sequence, then for
  *            kinds 0/1 first token and token count, for kind 2 stream blocks
  *            [x, y); flags (1 enters from a published state, 2 publishes its
  *            final state, 4 ends its sequence, 8 computes its local state
- *            first); entering slot and flag value; publishing slot and value.
+ *            first); entering slot and flag value; publishing slot and value (the
+ *            chunk scan's values are chunk numbers; a hand-over or split-scan
+ *            flag shows 1 here and carries a tag unique to the launch on the
+ *            device, so its scratch needs no zeroing).
  * Records are listed per CTA in processing order.  *n_rec receives the
  * number of records; returns LA_ERR_WORKSPACE (records beyond max_rec not
  * written) if max_rec is too small, LA_ERR_SHAPE / LA_ERR_NULL on bad

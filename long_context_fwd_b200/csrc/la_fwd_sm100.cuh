@@ -125,12 +125,12 @@ __device__ __forceinline__ bool get_item(const Params& p, const volatile uint32_
   return get_item(p, static_cast<int>(gridDim.x), static_cast<int>(blockIdx.x), m, w, it);
 }
 
-__device__ __forceinline__ void st_release_gpu(int* ptr, int v) {
-  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+__device__ __forceinline__ void st_release_gpu(unsigned long long* ptr, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(ptr), "l"(v) : "memory");
 }
-__device__ __forceinline__ int ld_acquire_gpu(const int* ptr) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* ptr) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ptr) : "memory");
   return v;
 }
 
@@ -921,8 +921,8 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
                                ? p.final_state + static_cast<int64_t>(it.seq) * state_elems + row_off
                                : nullptr;
     float* const pub_dst = it.publish ? p.prefix + static_cast<int64_t>(it.pub_slot) * (HD * HD) : nullptr;
-    int* const pub_flag = it.publish ? p.flags + it.pub_slot : nullptr;
-    const int pub_val = it.pub_val;
+    unsigned long long* const pub_flag = it.publish ? p.flags + it.pub_slot : nullptr;
+    const unsigned long long pub_val = it.pub_val;
     bool ok = true;
     for (int n = 0; n < it.nb && ok; ++n) {
       const uint32_t g = gb;

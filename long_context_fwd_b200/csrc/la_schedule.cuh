@@ -19,8 +19,11 @@ LA_HD T la_max(T a, T b) { return a < b ? b : a; }
 struct Params {
   const float* slopes;        // [H]
   float* prefix;              // [nseq][2][HD*HD] inclusive chunk states (chunked runs)
-  int* flags;                 // [nseq][2] publication flags (chunked runs), zeroed
-  int* ticket;                // work counter (chunked runs), zeroed
+  unsigned long long* flags;  // publication flags: the chunk scan's chunk numbers (zeroed
+                              // before the launch) or this launch's tag (hand-over, split scan)
+  int* ticket;                // work counter (chunk scan), zeroed before the launch
+  unsigned long long tag;     // nonzero and unique to the launch: the flag value the hand-over
+                              // and the split scan publish, so their flags need no zeroing
   const float* init_state;    // nullable [nseq][HD*HD]
   float* final_state;         // nullable [nseq][HD*HD]
   int* status;                // sticky error word
@@ -61,7 +64,8 @@ struct Item {
   bool publish;  // final state published after the outputs (balanced split)
   bool enter;    // starts from a published state: prefix[enter_slot] once flags[enter_slot] == enter_val
   bool last;     // ends its sequence (final state goes to the caller)
-  int enter_slot, enter_val, pub_slot, pub_val;
+  int enter_slot, pub_slot;
+  unsigned long long enter_val, pub_val;
 };
 
 // Ticket w of a chunked or unchunked run: chunk-major order, so every chunk of
@@ -79,9 +83,9 @@ LA_HD Item decode_item(const Params& p, int w) {
   it.enter = it.chunk > 0;
   it.last = it.chunk + 1 == p.nchunks;
   it.enter_slot = it.seq * 2 + ((it.chunk - 1) & 1);
-  it.enter_val = it.chunk;
+  it.enter_val = static_cast<unsigned long long>(it.chunk);
   it.pub_slot = it.seq * 2 + (it.chunk & 1);
-  it.pub_val = it.chunk + 1;
+  it.pub_val = static_cast<unsigned long long>(it.chunk) + 1u;
   return it;
 }
 
@@ -122,7 +126,7 @@ LA_HD bool balanced_item(const Params& p, int j, const volatile uint32_t* m, int
   it.publish = it.enter = false;
   it.enter_slot = j - 1;
   it.pub_slot = j;
-  it.enter_val = it.pub_val = 1;
+  it.enter_val = it.pub_val = p.tag;
   int i = k;
   if (head_len && i == 0) {
     seq = static_cast<int>(m[4]);
@@ -217,7 +221,7 @@ LA_HD bool split_scan_item(const Params& p, int i, const volatile uint32_t* m, i
   const int n1 = static_cast<int>(m[4]);
   int seq, blk0, blk1;
   it.publish = it.enter = it.last = false;
-  it.pub_val = it.enter_val = 1;
+  it.pub_val = it.enter_val = p.tag;
   it.enter_slot = 0;
   if (k < n1) {  // local state of one piece of this CTA's pass share
     const int x = static_cast<int>(m[5 + k]), y = static_cast<int>(m[6 + k]);

@@ -5,7 +5,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
+#include <random>
 
 #include "lightning_attn.h"
 #include "sm100_ptx.cuh"
@@ -88,18 +90,20 @@ struct Plan {
   size_t ctrl = 0, bytes = 0;  // scratch: ticket + flags, then 64 KiB chunk states
 };
 
+// Scratch control block: the ticket (padded to 8 bytes), then n 64-bit flags.
+size_t ctrl_bytes(size_t n_flags) { return (8 + n_flags * 8 + 255) / 256 * 256; }
+
 Plan make_plan(int nseq, int N, int sms, int chunk) {
   Plan pl;
   const int nblk = (N + 127) / 128;
   pl.nblk = nblk;
   const size_t state_bytes = 128 * 128 * sizeof(float);
-  auto round256 = [](size_t x) { return (x + 255) / 256 * 256; };
   if (chunk == 0 && nseq >= sms) {
     pl.mode = la::fwd::MODE_HANDOVER;
     pl.L = nblk * 128;
     pl.grid = sms;
     if (nseq % sms != 0) {  // some sequence crosses a CTA boundary
-      pl.ctrl = round256((static_cast<size_t>(sms) + 1) * sizeof(int));
+      pl.ctrl = ctrl_bytes(static_cast<size_t>(sms));
       pl.bytes = pl.ctrl + static_cast<size_t>(sms) * state_bytes;
     }
     return pl;
@@ -132,7 +136,7 @@ Plan make_plan(int nseq, int N, int sms, int chunk) {
       pl.F = static_cast<int>(F);
       pl.G2 = static_cast<int>(G2);
       pl.P = static_cast<long long>(nseq) * F;
-      pl.ctrl = round256((2 * static_cast<size_t>(sms) + 1) * sizeof(int));
+      pl.ctrl = ctrl_bytes(2 * static_cast<size_t>(sms));
       pl.bytes = pl.ctrl + 2 * static_cast<size_t>(sms) * state_bytes;
       return pl;
     }
@@ -153,7 +157,7 @@ Plan make_plan(int nseq, int N, int sms, int chunk) {
   pl.total = static_cast<long long>(nseq) * pl.nchunks;
   pl.grid = static_cast<int>(pl.total < sms ? pl.total : sms);
   if (pl.nchunks > 1) {
-    pl.ctrl = round256((static_cast<size_t>(nseq) * 2 + 1) * sizeof(int));
+    pl.ctrl = ctrl_bytes(static_cast<size_t>(nseq) * 2);
     pl.bytes = pl.ctrl + static_cast<size_t>(nseq) * 2 * state_bytes;
   }
   return pl;
@@ -174,8 +178,34 @@ void apply_plan(const Plan& pl, int nseq, la::fwd::Params& p) {
 
 void set_scratch(const Plan& pl, void* scratch, la::fwd::Params& p) {
   p.ticket = static_cast<int*>(scratch);
-  p.flags = p.ticket + 1;
+  p.flags = reinterpret_cast<unsigned long long*>(static_cast<char*>(scratch) + 8);
   p.prefix = reinterpret_cast<float*>(static_cast<char*>(scratch) + pl.ctrl);
+}
+
+// Only the chunk scan's ticket and flags (chunk numbers) need zeroing before a
+// launch; the hand-over and the split scan publish the launch's tag.
+bool needs_zeroed_ctrl(const Plan& pl) { return pl.mode == la::fwd::MODE_TICKETS; }
+
+// A nonzero 64-bit value unique to each launch of this process: the flag value
+// the hand-over and the split scan publish, so that scratch left by earlier
+// launches (or holding anything else) never reads as published.  SplitMix64
+// (Steele, Lea and Flood, "Fast splittable pseudorandom number generators",
+// OOPSLA 2014) of a per-process counter times an odd constant plus a random
+// seed: a bijection of the counter, so no two launches share a tag, and other
+// contents of the scratch match it with probability 2^-64 per flag read.
+unsigned long long launch_tag() {
+  static const unsigned long long seed = [] {
+    std::random_device rd;
+    return (static_cast<unsigned long long>(rd()) << 32) ^ rd();
+  }();
+  static std::atomic<unsigned long long> counter{0};
+  for (;;) {
+    unsigned long long z = seed + 0x9E3779B97F4A7C15ull * (counter.fetch_add(1) + 1);
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    z ^= z >> 31;
+    if (z != 0) return z;
+  }
 }
 
 // Element strides {b, h, t} of q, k, v and out (d or e contiguous).
@@ -326,14 +356,18 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   p.ticket_base = first_chunk * nseq;
   p.wait_limit_ns = wait_limit_ns;
 
+  p.tag = launch_tag();
+
   void* scratch = nullptr;
   if (pl.bytes) {
     cudaError_t e = cudaMallocAsync(&scratch, pl.bytes, stream);
     if (e != cudaSuccess) return cuda_fail(e);
-    e = cudaMemsetAsync(scratch, 0, pl.ctrl, stream);
-    if (e != cudaSuccess) {
-      cudaFreeAsync(scratch, stream);
-      return cuda_fail(e);
+    if (needs_zeroed_ctrl(pl)) {
+      e = cudaMemsetAsync(scratch, 0, pl.ctrl, stream);
+      if (e != cudaSuccess) {
+        cudaFreeAsync(scratch, stream);
+        return cuda_fail(e);
+      }
     }
     set_scratch(pl, scratch, p);
   }
@@ -414,14 +448,18 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
   p.N = N;
   apply_plan(pl, nseq, p);
   p.wait_limit_ns = kWaitLimitNs;
+  p.tag = launch_tag();
   if (pl.bytes) {
     void* scratch = nullptr;
     const int rc = noalloc_scratch_ptr(&scratch);
     if (rc != LA_OK) return rc;
-    // the array keeps the previous call's contents: the ticket and the flags
-    // must start at zero (the chunk states are always written before read)
-    const cudaError_t e = cudaMemsetAsync(scratch, 0, pl.ctrl, stream);
-    if (e != cudaSuccess) return cuda_fail(e);
+    // the array keeps the previous call's contents: the chunk scan's ticket
+    // and flags must start at zero (the chunk states are always written
+    // before they are read; the other splits' flags carry this launch's tag)
+    if (needs_zeroed_ctrl(pl)) {
+      const cudaError_t e = cudaMemsetAsync(scratch, 0, pl.ctrl, stream);
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
     set_scratch(pl, scratch, p);
   }
   return launch_fwd(rank, false, pl.grid, stream, tq, tk, tv, to, p);
@@ -576,7 +614,8 @@ int lightning_attn_fwd_plan(int B, int H, int N, int chunk, int sms, int* info, 
   info[4] = pl.F;
   info[5] = pl.G2;
   info[6] = static_cast<int>(pl.bytes > pl.ctrl ? (pl.bytes - pl.ctrl) / (128 * 128 * sizeof(float)) : 0);
-  info[7] = pl.ctrl ? static_cast<int>(pl.ctrl / sizeof(int)) - 1 : 0;
+  info[7] = pl.ctrl ? static_cast<int>((pl.ctrl - 8) / 8) : 0;
+  p.tag = 1;  // the records show the published flag value of a split as 1
   int n = 0;
   auto put = [&](int cta, int kind, int seq, int a, int b, int flags, int es, int ev, int ps,
                  int pv) {
@@ -590,8 +629,8 @@ int lightning_attn_fwd_plan(int B, int H, int N, int chunk, int sms, int* info, 
   auto put_item = [&](int cta, const la::fwd::Item& it) {
     const int flags = (it.enter ? 1 : 0) | (it.publish ? 2 : 0) | (it.last ? 4 : 0) |
                       (it.phase1 ? 8 : 0);
-    put(cta, it.p2 ? 0 : 1, it.seq, it.t0, it.Lc, flags, it.enter_slot, it.enter_val, it.pub_slot,
-        it.pub_val);
+    put(cta, it.p2 ? 0 : 1, it.seq, it.t0, it.Lc, flags, it.enter_slot,
+        static_cast<int>(it.enter_val), it.pub_slot, static_cast<int>(it.pub_val));
   };
   if (pl.mode == la::fwd::MODE_TICKETS) {
     for (int w = 0; w < static_cast<int>(pl.total); ++w) {

@@ -330,7 +330,7 @@ def device_status(reset: bool = True) -> int:
 
 PLAN_FIELDS = ("cta", "kind", "seq", "a", "b", "flags", "enter_slot", "enter_val", "pub_slot",
                "pub_val")
-PLAN_INFO = ("mode", "grid", "L", "nchunks", "F", "G2", "slots", "flag_words")
+PLAN_INFO = ("mode", "grid", "L", "nchunks", "F", "G2", "slots", "flags")
 
 
 def fwd_plan(B: int, H: int, N: int, chunk: int = 0, sms: int = 148):
