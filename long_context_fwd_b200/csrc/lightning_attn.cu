@@ -183,8 +183,15 @@ void set_scratch(const Plan& pl, void* scratch, la::fwd::Params& p) {
 }
 
 // Only the chunk scan's ticket and flags (chunk numbers) need zeroing before a
-// launch; the hand-over and the split scan publish the launch's tag.
-bool needs_zeroed_ctrl(const Plan& pl) { return pl.mode == la::fwd::MODE_TICKETS; }
+// launch; the hand-over and the split scan publish the launch's tag -- except
+// in a stream capture, where the tag is frozen into the graph and every replay
+// would find the previous replay's flags already set: there the captured
+// memset clears them (a zero flag never equals a tag).
+bool needs_zeroed_ctrl(const Plan& pl, cudaStream_t stream) {
+  if (pl.mode == la::fwd::MODE_TICKETS) return true;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  return cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone;
+}
 
 // A nonzero 64-bit value unique to each launch of this process: the flag value
 // the hand-over and the split scan publish, so that scratch left by earlier
@@ -362,7 +369,7 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   if (pl.bytes) {
     cudaError_t e = cudaMallocAsync(&scratch, pl.bytes, stream);
     if (e != cudaSuccess) return cuda_fail(e);
-    if (needs_zeroed_ctrl(pl)) {
+    if (needs_zeroed_ctrl(pl, stream)) {
       e = cudaMemsetAsync(scratch, 0, pl.ctrl, stream);
       if (e != cudaSuccess) {
         cudaFreeAsync(scratch, stream);
@@ -456,7 +463,7 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
     // the array keeps the previous call's contents: the chunk scan's ticket
     // and flags must start at zero (the chunk states are always written
     // before they are read; the other splits' flags carry this launch's tag)
-    if (needs_zeroed_ctrl(pl)) {
+    if (needs_zeroed_ctrl(pl, stream)) {
       const cudaError_t e = cudaMemsetAsync(scratch, 0, pl.ctrl, stream);
       if (e != cudaSuccess) return cuda_fail(e);
     }
