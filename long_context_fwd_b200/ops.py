@@ -8,6 +8,7 @@ functions: if the library is missing or a call fails, they raise.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import threading
 from typing import Optional
@@ -93,6 +94,29 @@ def _stream_handle(stream: Optional[torch.cuda.Stream]) -> int:
     return int(s.cuda_stream)
 
 
+def _on_tensor_device(fn):
+    """Runs an entry point on the CUDA device its tensors live on (the library
+    launches on the calling thread's current device, with that device's
+    current stream by default); tensors on different devices are refused, so
+    no kernel is ever handed another device's pointers."""
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        tensors = [a for a in (*args, *kwargs.values()) if isinstance(a, torch.Tensor)]
+        devices = {t.device for t in tensors if t.is_cuda}
+        if len(devices) > 1:
+            raise ValueError(f"{fn.__name__}: all tensors must be on one CUDA device, got "
+                             f"{sorted(str(d) for d in devices)}")
+        if not devices:
+            return fn(*args, **kwargs)  # the argument checks reject non-CUDA tensors
+        (dev,) = devices
+        stream = kwargs.get("stream")
+        if stream is not None and stream.device != dev:
+            raise ValueError(f"{fn.__name__}: stream is on {stream.device}, tensors on {dev}")
+        with torch.cuda.device(dev):
+            return fn(*args, **kwargs)
+    return wrapper
+
+
 def _need(t: torch.Tensor, name: str, dtype, shape):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -106,6 +130,7 @@ def _need(t: torch.Tensor, name: str, dtype, shape):
         raise ValueError(f"{name} must be contiguous")
 
 
+@_on_tensor_device
 def fwd(q, k, v, slopes, out=None, *, init_state=None, final_state=None, chunk: int = 0,
         stream=None) -> torch.Tensor:
     """Prefill: bf16 q, k [B,H,N,D], v [B,H,N,E], fp32 slopes [H] -> fp32 out [B,H,N,E]."""
@@ -149,6 +174,7 @@ def _need_view(t: torch.Tensor, name: str, dtype, shape):
         raise ValueError(f"{name}: the last dimension must be contiguous")
 
 
+@_on_tensor_device
 def fwd_strided(q, k, v, slopes, out, *, init_state=None, final_state=None, chunk: int = 0,
                 stream=None) -> torch.Tensor:
     """Prefill on strided views: q, k [B,H,N,D] and v [B,H,N,E] bf16, out [B,H,N,E] fp32,
@@ -176,6 +202,7 @@ def fwd_strided(q, k, v, slopes, out, *, init_state=None, final_state=None, chun
     return out
 
 
+@_on_tensor_device
 def fwd_anticausal(q, k, v, slopes, out=None, *, init_state=None, final_state=None,
                    chunk: int = 0, stream=None) -> torch.Tensor:
     """Anti-causal prefill, o_t = sum_{s >= t} g^(s-t) (q_t . k_s) v_s (shapes as fwd)."""
@@ -200,6 +227,7 @@ def fwd_anticausal(q, k, v, slopes, out=None, *, init_state=None, final_state=No
     return out
 
 
+@_on_tensor_device
 def fwd_fused(q, k, v, gate, slopes, norm_weight, eps: float = 1e-6, out=None, *,
               stream=None) -> torch.Tensor:
     """The fused layer: raw bf16 q, k [B,H,N,D], v, gate [B,H,N,E], fp32 norm_weight
@@ -222,6 +250,7 @@ def fwd_fused(q, k, v, gate, slopes, norm_weight, eps: float = 1e-6, out=None, *
     return out
 
 
+@_on_tensor_device
 def bwd(q, k, v, dout, slopes, dq=None, dk=None, dv=None, *, stream=None):
     """Backward pass: bf16 q, k [B,H,N,D], v, dout [B,H,N,E] -> fp32 (dq, dk, dv)."""
     B, H, N, D = q.shape
@@ -244,6 +273,7 @@ def bwd(q, k, v, dout, slopes, dq=None, dk=None, dv=None, *, stream=None):
     return dq, dk, dv
 
 
+@_on_tensor_device
 def fwd_noalloc(q, k, v, slopes, out=None, *, chunk: int = 0, stream=None) -> torch.Tensor:
     """Prefill through the allocation-free entry point (scratch in a fixed device array).
 
@@ -268,6 +298,7 @@ def fwd_noalloc(q, k, v, slopes, out=None, *, chunk: int = 0, stream=None) -> to
     return out
 
 
+@_on_tensor_device
 def fwd_f32(q, k, v, slopes, out=None, *, stream=None) -> torch.Tensor:
     """Prefill with fp32 q, k, v -> fp32 out."""
     B, H, N, D = q.shape
@@ -285,6 +316,7 @@ def fwd_f32(q, k, v, slopes, out=None, *, stream=None) -> torch.Tensor:
     return out
 
 
+@_on_tensor_device
 def decode(q, k, v, state, slopes, out=None, *, stream=None) -> torch.Tensor:
     """One decode step: bf16 q, k [B,H,D], v [B,H,E]; fp32 state [B,H,D,E] in place."""
     B, H, D = q.shape
@@ -304,6 +336,7 @@ def decode(q, k, v, state, slopes, out=None, *, stream=None) -> torch.Tensor:
     return out
 
 
+@_on_tensor_device
 def fault_test_scan_stall(q, k, v, slopes, out, *, chunk: int, wait_limit_ms: int,
                           stream=None) -> None:
     """Runs the prefill with chunk 0 never processed (see the C header): every

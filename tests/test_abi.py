@@ -96,6 +96,20 @@ def test_binding_rejects_cpu_tensors():
         ops.fwd(x, x, x, torch.zeros(1))
 
 
+def test_binding_runs_each_entry_on_its_tensors_device():
+    # every entry point is wrapped so it launches on the device of its tensors
+    # and refuses tensors spread over devices (checked with real devices on GPU
+    # boxes; here the wrapper's pass-through for non-CUDA tensors)
+    for name in ("fwd", "fwd_strided", "fwd_anticausal", "fwd_fused", "bwd", "fwd_noalloc",
+                 "fwd_f32", "decode", "fault_test_scan_stall"):
+        fn = getattr(ops, name)
+        assert getattr(fn, "__wrapped__", None) is not None, name
+    import torch
+    x = torch.zeros((1, 1, 4, 64))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ops.fwd_f32(x, x, x, torch.zeros(1))
+
+
 def test_fault_hook_validation(lib):
     f = lib.lightning_attn_fault_test_scan_stall
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1024, 0, 100, None) == LA_ERR_SHAPE
