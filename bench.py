@@ -42,12 +42,23 @@ KERNEL_SOURCES = ("long_context_fwd_b200/csrc/la_fwd_sm100.cuh",
 PROFILE = os.path.join(ROOT, "profiles", "prefill_bf16_tcgen05.md")
 
 
+def _code_only(text: str) -> str:
+    """C++ source with comments and blank lines removed, lines right-stripped
+    (string literals in the kernel sources hold no comment markers)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_hash() -> str:
+    """sha256 (first 16 hex) of the prefill kernel's code: a comment edit keeps
+    the committed ncu capture valid, any code change invalidates it."""
     import hashlib
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f)) as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -14,16 +14,25 @@
 //   S   <- gamma^len S + (gamma^(len-1-j) K)^T V   (tensor cores, fp32 in TMEM)
 // Every decay factor used is gamma^m with 0 <= m <= 128, so nothing overflows.
 //
-// Sequence split (chunked scan).  To give all SMs work when B*H is small, a
-// sequence is cut into chunks of L tokens (L a multiple of 128).  Work item
-// w = chunk * (B*H) + seq.  A chunk with a successor first computes its local
-// state A_c = sum_j gamma^(Lc-1-j) k_j^T v_j over its tokens (phase 1, K/V
-// kept in L2 with an evict-last hint), then takes the inclusive state of the
-// previous chunk from global memory (spin on a flag, bounded in time),
-// publishes its own inclusive state gamma^Lc S_prev + A_c, and runs the
-// blocked form from S_prev (phase 2, re-reading K/V from L2).  Items are handed
-// out through an atomic ticket, so every chunk's predecessor is held by a CTA
-// that is already running: no co-residency assumption.
+// Work splits (the items of each CTA are computed in la_schedule.cuh):
+//   * whole sequences, or a balanced hand-over when B*H >= SMs (a sequence cut
+//     between two CTAs: the first part publishes its final state, the second
+//     part runs last and starts from it);
+//   * the split scan when SMs/8 <= B*H < SMs (a local-state pass over the first
+//     parts of all sequences, cut into pieces; a share that starts inside a
+//     sequence adds up the pieces before it);
+//   * the chunked scan otherwise.  Work item w = chunk * (B*H) + seq.  A chunk
+//     with a successor first computes its local state A_c = sum_j
+//     gamma^(Lc-1-j) k_j^T v_j over its tokens (phase 1, K/V kept in L2 with an
+//     evict-last hint), then takes the inclusive state of the previous chunk
+//     from global memory (spin on a flag, bounded in time), publishes its own
+//     inclusive state gamma^Lc S_prev + A_c, and runs the blocked form from
+//     S_prev (phase 2).  Items are handed out through an atomic ticket, so every
+//     chunk's predecessor is held by a CTA that is already running: no
+//     co-residency assumption.
+// Published states are 64 KiB fp32 in scratch with a 64-bit flag stored with
+// release semantics; the hand-over and the split scan publish a value unique
+// to the launch, so their flags need no clearing between launches.
 //
 // Roles (448 threads, one CTA per SM):
 //   warps 0..7   group X: decay-causal mask of Q K^T into P (bf16, TMEM),
@@ -34,7 +43,9 @@
 //                the epilogue (TMEM -> swizzled shared memory -> TMA store).
 //                Thread t owns row r = 32 (warp % 4) + lane, all 128 columns.
 //   warp 12      TMA producer: Q/K/V tiles into three 2-slot rings.
-//   warp 13      TMEM allocator and single-thread tcgen05.mma issuer.
+//   warp 13      TMEM allocator and single-thread tcgen05.mma issuer: per block
+//                the state update, inter and intra products, then the next
+//                block's Q K^T (which waits for the next K tile).
 // X and Y run concurrently on different blocks' data.
 // TMEM (512 columns): S/P double buffer [0,256), O [256,384), state [384,512).
 // After group X has read the scores of an S buffer it rewrites the buffer with

@@ -52,3 +52,10 @@ def test_other_split_counts_and_stale_captures_give_none(current, monkeypatch):
     assert bench.measured_traffic(I.Workload("x", 1, 32, 65536, 128, 128, "bf16", index=950), 148) is None
     monkeypatch.setattr(bench, "kernel_hash", lambda: "0" * 16)
     assert bench.measured_traffic(I.PREFILL_32K, 148) is None
+
+
+def test_kernel_hash_ignores_comments_only():
+    code = "int f(int x) {  // doubles\n  /* a block\n comment */ return 2 * x;\n}\n\n"
+    assert bench._code_only(code) == "int f(int x) {\n   return 2 * x;\n}"
+    assert bench._code_only(code.replace("doubles", "twice")) == bench._code_only(code)
+    assert bench._code_only(code.replace("2 * x", "3 * x")) != bench._code_only(code)
