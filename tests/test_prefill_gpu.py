@@ -116,6 +116,8 @@ MANY_SEQ_CASES = [
     (1, 149, 1025, 0),
     (1, 296, 300, 0),
     (2, 80, 1100, 256),
+    (16, 64, 200, 0),    # 1024 short sequences, about 7 per SM with a hand-over each
+    (8, 64, 129, 0),     # one token past a block
 ]
 
 
