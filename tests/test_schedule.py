@@ -18,6 +18,7 @@ SM counts:
 """
 import collections
 
+import numpy as np
 import pytest
 
 from long_context_fwd_b200 import build, ops
@@ -76,17 +77,17 @@ def test_every_output_once(B, H, N, sms):
     assert info["grid"] <= sms
 
 
-@pytest.mark.parametrize("B,H,N,chunk", [(1, 4, 3000, 512), (3, 4, 2100, 128), (2, 80, 1100, 256),
-                                         (1, 2, 4097, 1024), (1, 64, 8192, 2048)])
-def test_explicit_chunks_use_the_chunk_scan(B, H, N, chunk):
-    info, items = _plan(B, H, N, chunk)
-    assert info["mode"] == 0 and info["L"] == chunk
+def _check_chunk_scan(B, H, N, info, items):
+    """Chunk scan: ticket w is chunk w // (B*H) of sequence w % (B*H); every
+    chunk once; each waits for its predecessor's value in the alternate slot
+    and publishes its own."""
+    assert info["mode"] == 0
     _check_outputs(B, H, N, items)
-    nseq, nch = B * H, info["nchunks"]
+    nseq, nch, L = B * H, info["nchunks"], info["L"]
     seen = set()
     for w, it in enumerate(items):
         c = w // nseq
-        assert it["cta"] == -1 and it["seq"] == w % nseq and it["a"] == c * chunk
+        assert it["cta"] == -1 and it["seq"] == w % nseq and it["a"] == c * L
         seen.add((it["seq"], c))
         assert bool(it["flags"] & PHASE1) == (c + 1 < nch)
         if c > 0:
@@ -97,6 +98,14 @@ def test_explicit_chunks_use_the_chunk_scan(B, H, N, chunk):
     assert len(seen) == nseq * nch
 
 
+@pytest.mark.parametrize("B,H,N,chunk", [(1, 4, 3000, 512), (3, 4, 2100, 128), (2, 80, 1100, 256),
+                                         (1, 2, 4097, 1024), (1, 64, 8192, 2048)])
+def test_explicit_chunks_use_the_chunk_scan(B, H, N, chunk):
+    info, items = _plan(B, H, N, chunk)
+    assert info["L"] == chunk
+    _check_chunk_scan(B, H, N, info, items)
+
+
 def _per_cta(items):
     by = collections.defaultdict(list)
     for it in items:
@@ -104,11 +113,10 @@ def _per_cta(items):
     return by
 
 
-@pytest.mark.parametrize("sms", [148, 132])
-@pytest.mark.parametrize("B,H,N", [(4, 64, 32768), (1, 149, 1025), (2, 80, 1100), (1, 150, 2500),
-                                   (1, 296, 300), (3, 100, 700), (1, 200, 5000)])
-def test_balanced_handover(B, H, N, sms):
-    info, items = _plan(B, H, N, sms=sms)
+def _check_handover(B, H, N, sms, info, items):
+    """Balanced hand-over: equal block shares; a publishing item runs first on
+    its CTA, its sequence's entering item last on the next CTA, starting where
+    it ends."""
     assert info["mode"] == 1 and info["grid"] == sms
     by = _per_cta(items)
     nblk = -(-N // BLK)
@@ -129,6 +137,14 @@ def test_balanced_handover(B, H, N, sms):
         assert info["slots"] == 0 and not any(it["flags"] & (ENTER | PUBLISH) for it in items)
 
 
+@pytest.mark.parametrize("sms", [148, 132])
+@pytest.mark.parametrize("B,H,N", [(4, 64, 32768), (1, 149, 1025), (2, 80, 1100), (1, 150, 2500),
+                                   (1, 296, 300), (3, 100, 700), (1, 200, 5000)])
+def test_balanced_handover(B, H, N, sms):
+    info, items = _plan(B, H, N, sms=sms)
+    _check_handover(B, H, N, sms, info, items)
+
+
 @pytest.mark.parametrize("sms", [148, 132, 160])
 @pytest.mark.parametrize("B,H,N", [(1, 64, 8192), (1, 64, 1048576), (1, 19, 3000), (1, 37, 1025),
                                    (1, 100, 2000), (1, 147, 1200), (1, 64, 1152),
@@ -144,6 +160,15 @@ def test_split_scan(B, H, N, sms):
         ok_whole = nblk <= 8 or nseq * nblk / sms > 0.6 * nblk
         assert 8 * nseq < sms or ok_whole, info
         return
+    _check_split_scan(B, H, N, sms, info, items)
+
+
+def _check_split_scan(B, H, N, sms, info, items):
+    """Split scan: local-state items partition the first F blocks of every
+    sequence in distinct slots; each entering state chains exactly the pieces
+    before it, in order; both passes balanced; never slower than one whole
+    sequence per SM."""
+    nseq, nblk = B * H, -(-N // BLK)
     assert info["mode"] == 2, info
     F, G2, G = info["F"], info["G2"], info["grid"]
     assert G == sms and G2 == sms - nseq and 1 <= F < nblk
@@ -224,3 +249,39 @@ def test_plan_rejects_bad_arguments():
     # too small a record buffer reports the count and LA_ERR_WORKSPACE
     assert lib.lightning_attn_fwd_plan(1, 64, 8192, 0, 148, info, None, 0, ctypes.byref(n)) == 7
     assert n.value > 0
+
+
+def _random_shapes(n, seed):
+    """Seeded shapes over every work split: many sequences (hand-over), the
+    split-scan range, few sequences (chunk scan or whole sequences), lengths
+    log-uniform from 1 token to 128K, several SM counts."""
+    rng = np.random.default_rng(seed)
+    for _ in range(n):
+        sms = int(rng.choice([148, 132, 160, 114, 80, 8]))
+        pick = int(rng.integers(3))
+        if pick == 0:
+            nseq = int(rng.integers(sms, 6 * sms))
+        elif pick == 1:
+            nseq = int(rng.integers(max(1, sms // 8), sms))
+        else:
+            nseq = int(rng.integers(1, max(2, sms // 8)))
+        B = int(rng.choice([d for d in range(1, 9) if nseq % d == 0]))
+        N = int(rng.integers(1, 1 << int(rng.integers(1, 18))))
+        yield B, nseq // B, N, sms
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_random_shapes_keep_every_invariant(seed):
+    modes = collections.Counter()
+    for B, H, N, sms in _random_shapes(60, seed):
+        info, items = _plan(B, H, N, sms=sms)
+        modes[info["mode"]] += 1
+        _check_outputs(B, H, N, items)
+        assert info["grid"] <= sms
+        if info["mode"] == 1:
+            _check_handover(B, H, N, sms, info, items)
+        elif info["mode"] == 2:
+            _check_split_scan(B, H, N, sms, info, items)
+        else:
+            _check_chunk_scan(B, H, N, info, items)
+    assert len(modes) == 3, modes  # the draw reaches every split
