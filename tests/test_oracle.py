@@ -60,6 +60,28 @@ def test_forms_match_bruteforce(B, H, N, D, E, slopes):
         assert _rel(out, ref) <= 1e-12, name
 
 
+@pytest.mark.parametrize("seed", range(6))
+def test_forms_match_bruteforce_random_shapes(seed):
+    """Seeded random shapes, slopes (including 0 and large) and block sizes:
+    every C form against the pure-Python brute force."""
+    rng = np.random.default_rng(700 + seed)
+    B, H = int(rng.integers(1, 3)), int(rng.integers(1, 4))
+    N, D, E = int(rng.integers(1, 48)), int(rng.integers(1, 10)), int(rng.integers(1, 10))
+    slopes = [float(x) for x in rng.choice([0.0, 0.01, 0.3, 1.0, 4.0], size=H)]
+    q, k, v = (_rand((B, H, N, n), 10 * seed + i, scale) for i, (n, scale) in
+               enumerate(((D, 1.0), (D, 0.5), (E, 2.0))))
+    ref = np.zeros((B, H, N, E))
+    for b in range(B):
+        for h in range(H):
+            ref[b, h] = np.array(brute_force(q[b, h], k[b, h], v[b, h],
+                                             float(np.float32(slopes[h])))).reshape(N, E)
+    forms = {"masked": oracle.masked(q, k, v, slopes), "recurrent": oracle.recurrent(q, k, v, slopes)}
+    for blk in {1, int(rng.integers(1, N + 1)), N}:
+        forms[f"blocked{blk}"] = oracle.blocked(q, k, v, slopes, blk)
+    for name, out in forms.items():
+        assert _rel(out, ref) <= 1e-12, (name, B, H, N, D, E, slopes)
+
+
 @pytest.mark.parametrize("lam", [0.0, 0.05, 0.7, 2.0])
 def test_closed_form_unit_inputs(lam):
     # D = E = 1, q = k = v = 1: o_t = sum_{s<=t} gamma^(t-s) = (1 - gamma^(t+1)) / (1 - gamma),
