@@ -112,8 +112,10 @@ int lightning_attn_fwd_ex(const void* q, const void* k, const void* v,
  *
  *   q, k, v, slopes, out, B, H, N, D, E, stream: as lightning_attn_fwd.
  *   chunk: as lightning_attn_fwd_ex (0 = automatic).
- * Scratch needed when the sequences are split: 256-byte-rounded
- * (2 B H + 1) * 4 bytes of counters plus B H * 128 KiB of chunk states.  A call
+ * Scratch needed when the sequences are split: a 256-byte-rounded control
+ * block (an 8-byte ticket and one 64-bit flag per state slot) plus 64 KiB per
+ * state slot -- 2 B H slots for the chunk scan, at most 2 per SM for the
+ * automatic splits.  A call
  * that would need more than LA_NOALLOC_SCRATCH_BYTES returns LA_ERR_WORKSPACE
  * before launching anything.  With chunk = 0 the split is only used when B*H
  * is below the SM count, which stays within the limit on a 148-SM B200.
