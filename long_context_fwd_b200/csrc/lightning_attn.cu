@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <chrono>
 #include <mutex>
 #include <random>
 
@@ -202,8 +203,18 @@ bool needs_zeroed_ctrl(const Plan& pl, cudaStream_t stream) {
 // contents of the scratch match it with probability 2^-64 per flag read.
 unsigned long long launch_tag() {
   static const unsigned long long seed = [] {
-    std::random_device rd;
-    return (static_cast<unsigned long long>(rd()) << 32) ^ rd();
+    // the C ABI never throws: without an entropy source, the clock and an
+    // address of this process seed it (distinct launches still get distinct
+    // tags; only foreign scratch contents would be less unpredictable)
+    unsigned long long z = static_cast<unsigned long long>(
+        std::chrono::high_resolution_clock::now().time_since_epoch().count());
+    z ^= reinterpret_cast<uintptr_t>(&z);
+    try {
+      std::random_device rd;
+      z ^= (static_cast<unsigned long long>(rd()) << 32) ^ rd();
+    } catch (...) {
+    }
+    return z;
   }();
   static std::atomic<unsigned long long> counter{0};
   for (;;) {
