@@ -32,7 +32,6 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "lightning-attn prefill tokens/s (% roofline); decode tokens/s (HBM GB/s)"
-BYTES_PER_TOKEN_HEAD = 2 * 128 + 2 * 128 + 2 * 128 + 4 * 128  # q, k, v bf16 in + out fp32
 BLK = 128  # tokens per block in the prefill kernel
 
 
@@ -126,6 +125,15 @@ def parse():
                     help="steps of the backward-pass leg (0 skips it)")
     ap.add_argument("--fused-steps", type=int, default=20,
                     help="steps of the fused-layer leg (0 skips it)")
+    ap.add_argument("--sustained-steps", type=int, default=1000,
+                    help="a second timing of the headline workload over this many launches "
+                         "(clocks settled under the power cap; 0 skips it)")
+    ap.add_argument("--extra-workloads",
+                    default="prefill_b1h64n8192d128,prefill_b1h64n1048576d128",
+                    help="comma-separated prefill workloads timed as legs of the same line")
+    ap.add_argument("--extra-seconds", type=float, default=0.5,
+                    help="about this much roofline time per extra leg")
+    ap.add_argument("--extra-max-steps", type=int, default=300)
     return ap.parse_args()
 
 
@@ -192,15 +200,16 @@ class ClockSampler:
         self.windows.append((t0, t1))
 
     def stop(self):
+        """Ends sampling and parses the samples; summary() then reads them."""
+        self.rows = []
         if self.proc is None:
-            return None
+            return
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.tmp.flush()
-        rows = []
         with open(self.tmp.name) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
@@ -209,11 +218,17 @@ class ClockSampler:
                 try:
                     ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
                     ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
-                    rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
+                    self.rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
                 except (ValueError, IndexError, OverflowError):
                     continue
         os.unlink(self.tmp.name)
-        inside = [r for r in rows if any(a - 0.05 <= r[0] <= b + 0.05 for a, b in self.windows)]
+
+    def summary(self, windows=None):
+        """Median SM clock, max clock and active throttle reasons of the samples
+        taken inside `windows` (host-time intervals; default: every marked one)."""
+        rows = getattr(self, "rows", [])
+        windows = self.windows if windows is None else windows
+        inside = [r for r in rows if any(a - 0.05 <= r[0] <= b + 0.05 for a, b in windows)]
         use = inside if inside else rows[-5:]
         if not use:
             return None
@@ -223,9 +238,78 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(use), "in_timed_region": bool(inside)}
 
 
+def roofline(bytes_launch: float, flops_launch: float, kernel_ms: float, hbm: float,
+             tensor_peak: float, traffic=None, peak_src: str = "measured") -> dict:
+    """Roofline of one launch: the bound is the slower of its algorithmic bytes
+    at the HBM copy bandwidth and its algorithmic flops at the dense bf16
+    tensor peak; achieved and peak are given in the bound's unit and frac is
+    that lower-bound time over the measured launch time."""
+    t_bytes = bytes_launch / (hbm * 1e9)
+    t_flops = flops_launch / (tensor_peak * 1e12)
+    secs = kernel_ms / 1e3
+    if t_bytes >= t_flops:
+        r = {"bound": "hbm", "achieved": bytes_launch / secs / 1e9, "peak": hbm, "unit": "GB/s"}
+    else:
+        r = {"bound": "tensor", "achieved": flops_launch / secs / 1e12, "peak": tensor_peak,
+             "unit": "TFLOP/s"}
+    r.update({"frac": max(t_bytes, t_flops) / secs, "traffic": traffic,
+              "peak_source": f"{peak_src} ({'copy bandwidth' if r['bound'] == 'hbm' else 'bf16 GEMM'})",
+              "bytes_per_launch": bytes_launch, "flops_per_launch": flops_launch,
+              "kernel_ms": kernel_ms, "hbm_bound_ms": t_bytes * 1e3,
+              "tensor_bound_ms": t_flops * 1e3,
+              "tensor_tflops": flops_launch / secs / 1e12})
+    return r
+
+
 # ----------------------------------------------------------------------------
 # our implementation
 # ----------------------------------------------------------------------------
+def timed_launches(dist, stream, steps: int, fn) -> dict:
+    """Times `steps` calls of fn back to back with CUDA events on `stream`
+    (a barrier and a device synchronisation on both sides; the slowest rank's
+    times): the whole region and the mean per call."""
+    import torch
+    from long_context_fwd_b200 import ops
+
+    dist.barrier()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    t_host0 = time.time()
+    for i in range(steps):
+        starts[i].record(stream)
+        fn()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.time()
+    dist.barrier()
+    total_ms = starts[0].elapsed_time(ends[-1])
+    launch_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    return {"total_ms": dist.max(total_ms), "launch_ms": dist.max(launch_ms), "steps": steps,
+            "window": (t_host0, t_host1), "status": ops.device_status(reset=True)}
+
+
+def bench_prefill_leg(dist, w, dev, steps: int, warmup: int) -> dict:
+    """One more prefill workload timed on its own (inputs resident on the
+    device, head-major, automatic work split): a leg of the JSON line."""
+    import torch
+    from long_context_fwd_b200 import inputs as I
+    from long_context_fwd_b200 import ops
+
+    q, k, v = I.device_prefill_inputs(w, dev)
+    sl = torch.from_numpy(I.slopes_for(w)).to(dev)
+    out = torch.empty((w.B, w.H, w.N, w.E), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, warmup)):
+        ops.fwd(q, k, v, sl, out)
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0, "device-side wait timed out during warm-up"
+    res = timed_launches(dist, stream, steps, lambda: ops.fwd(q, k, v, sl, out))
+    del q, k, v, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_prefill(args, dist, w, dev):
     import torch
     from long_context_fwd_b200 import inputs as I
@@ -254,23 +338,12 @@ def bench_prefill(args, dist, w, dev):
         call(q, k, v, out)
     torch.cuda.synchronize()
     assert ops.device_status(reset=True) == 0, "device-side wait timed out during warm-up"
-    dist.barrier()
-    torch.cuda.synchronize()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    t_host0 = time.time()
-    for i in range(args.steps):
-        starts[i].record(stream)
-        call(q, k, v, out)
-        ends[i].record(stream)
-    torch.cuda.synchronize()
-    t_host1 = time.time()
-    dist.barrier()
-    total_ms = starts[0].elapsed_time(ends[-1])
-    launch_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
-    status = ops.device_status(reset=True)
-    res = {"total_ms": dist.max(total_ms), "launch_ms": dist.max(launch_ms),
-           "window": (t_host0, t_host1), "status": status}
+    res = timed_launches(dist, stream, args.steps, lambda: call(q, k, v, out))
+    if args.sustained_steps > 0:
+        # the same launches again, back to back for long enough that the
+        # clocks settle under the power cap
+        res["sustained"] = timed_launches(dist, stream, args.sustained_steps,
+                                          lambda: call(q, k, v, out))
     if args.e2e_steps <= 0:
         res["e2e_ms"], res["h2d"], res["d2h"] = None, 0, 0
         del q, k, v, out
@@ -387,8 +460,8 @@ def bench_decode(args, dist, dev):
     finite = bool(torch.isfinite(state).all().item())
     del qs, ks, vs, state
     torch.cuda.empty_cache()
-    return {"ms": ms, "bytes": bytes_step, "steps": steps, "window": (t_host0, t_host1),
-            "finite": finite, "workload": w.name, "tokens": w.B}
+    return {"ms": ms, "bytes": bytes_step, "flops": w.B * w.H * 5 * w.D * w.E, "steps": steps,
+            "window": (t_host0, t_host1), "finite": finite, "workload": w.name, "tokens": w.B}
 
 
 def bench_backward(args, dist, w, dev):
@@ -427,7 +500,12 @@ def bench_backward(args, dist, w, dev):
     status = ops.device_status(reset=True)
     del q, k, v, dout, dq, dk, dv
     torch.cuda.empty_cache()
-    return {"ms": ms, "steps": steps, "window": (t_host0, t_host1), "status": status}
+    units = w.B * w.H * w.N
+    # three launches, each reading three bf16 operands and writing fp32
+    moved = units * (2 * (2 * w.E + w.D) + 4 * w.D + 2 * (2 * w.D + w.E) + 4 * w.D +
+                     2 * (2 * w.D + w.E) + 4 * w.E)
+    return {"ms": ms, "steps": steps, "window": (t_host0, t_host1), "status": status,
+            "launches": 3, "bytes_moved": moved}
 
 
 def bench_fused(args, dist, w, dev):
@@ -455,17 +533,19 @@ def bench_fused(args, dist, w, dev):
     dist.barrier()
     steps = args.fused_steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_host0 = time.time()
     e0.record(stream)
     for _ in range(steps):
         ops.fwd_fused(q, k, v, gate, sl, nw, 1e-6, out)
     e1.record(stream)
     torch.cuda.synchronize()
+    t_host1 = time.time()
     dist.barrier()
     ms = dist.max(e0.elapsed_time(e1)) / steps
     status = ops.device_status(reset=True)
     del q, k, v, gate, out
     torch.cuda.empty_cache()
-    return {"ms": ms, "steps": steps, "status": status}
+    return {"ms": ms, "steps": steps, "status": status, "window": (t_host0, t_host1)}
 
 
 def cpu_baseline(w, seconds: float):
@@ -506,32 +586,51 @@ def job_throughput(world: int, units_per_rank: int, ms_per_step_max: float) -> f
     return world * units_per_rank / (ms_per_step_max / 1e3)
 
 
+def prefill_flops(w) -> int:
+    """Algorithmic flops of one prefill launch of the blocked form at the
+    kernel's 128-token blocks: 4 D E + 2 BLK (D + E) per token-head."""
+    return w.B * w.H * w.N * (4 * w.D * w.E + 2 * BLK * (w.D + w.E))
+
+
+def prefill_bytes(w) -> int:
+    """Algorithmic bytes of one prefill launch: q, k, v read once (bf16), out
+    written once (fp32)."""
+    return w.B * w.H * w.N * (2 * (w.D + w.D + w.E) + 4 * w.E)
+
+
 def main_ours(args):
     import torch
     from long_context_fwd_b200 import inputs as I
+    from long_context_fwd_b200 import ops
 
     dist = Dist()
     torch.cuda.set_device(dist.local)
     dev = torch.device("cuda", dist.local)
     dist.init("nccl")
     w = I.WORKLOADS[args.workload]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     hbm, bf16, bf16_sustained, peak_src = peaks()
     sampler = ClockSampler(dist.local)
     pre = bench_prefill(args, dist, w, dev)
-    sampler.mark(*pre["window"])
+    legs = {}
+    for name in [x for x in args.extra_workloads.split(",") if x]:
+        wx = I.WORKLOADS[name]
+        steps = max(3, min(args.extra_max_steps, int(args.extra_seconds * 1e3 /
+                                                    max(1e-3, prefill_bytes(wx) / hbm / 1e6))))
+        legs[name] = (wx, bench_prefill_leg(dist, wx, dev, steps, args.warmup))
     dec = None if args.no_decode else bench_decode(args, dist, dev)
     bwd = None if args.backward_steps <= 0 else bench_backward(args, dist, w, dev)
     fus = None if args.fused_steps <= 0 else bench_fused(args, dist, w, dev)
-    clocks = sampler.stop()
+    sampler.stop()
     tokens_step = w.B * w.N
     ms_step = pre["total_ms"] / args.steps
     value = job_throughput(dist.world, tokens_step, ms_step)
-    bytes_launch = w.B * w.H * w.N * BYTES_PER_TOKEN_HEAD
-    achieved = bytes_launch / (pre["launch_ms"] / 1e3) / 1e9
-    flops_launch = w.B * w.H * w.N * (4 * w.D * w.E + 2 * BLK * (w.D + w.E))
-    # the committed capture is of head-major tensors
-    traffic = (measured_traffic(w, torch.cuda.get_device_properties(dev).multi_processor_count)
-               if args.layout == "head-major" else None)
+    bytes_launch = prefill_bytes(w)
+
+    def traffic_for(wx):
+        # the committed captures are of head-major tensors
+        return measured_traffic(wx, sms) if args.layout == "head-major" else None
+
     line = {
         "metric": METRIC,
         "value": value,
@@ -551,12 +650,9 @@ def main_ours(args):
                    "parallelism": f"replicas x{dist.world} (independent (b,h) problems, no collective)",
                    "l2": f"no flush: each step streams {bytes_launch / 1e9:.2f} GB, larger than the "
                          "126 MB L2"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": traffic,
-                     "peak_source": f"{peak_src} copy bandwidth",
-                     "bytes_per_launch": bytes_launch, "kernel_ms": pre["launch_ms"],
-                     "tensor_tflops": flops_launch / (pre["launch_ms"] / 1e3) / 1e12,
-                     "tensor_peak_tflops": bf16, "tensor_peak_tflops_sustained": bf16_sustained},
+        "roofline": dict(roofline(bytes_launch, prefill_flops(w), pre["launch_ms"], hbm, bf16,
+                                  traffic_for(w), peak_src),
+                         tensor_peak_tflops_sustained=bf16_sustained),
         "gpu_launches": args.steps,
         "device_status": pre["status"],
         "e2e": None if pre["e2e_ms"] is None else {
@@ -565,42 +661,67 @@ def main_ours(args):
             "ms_per_step": pre["e2e_ms"],
             "pipelining": f"{pre['e2e_groups']} groups of sequences: uploads, prefills and "
                           "downloads on three streams, ordered per group by events"},
-        "clocks": clocks,
+        "clocks": sampler.summary([pre["window"]]),
     }
+    if "sustained" in pre:
+        su = pre["sustained"]
+        ck = sampler.summary([su["window"]])
+        line["sustained"] = {
+            "what": f"the headline launches again, {su['steps']} back to back",
+            "value": job_throughput(dist.world, tokens_step, su["total_ms"] / su["steps"]),
+            "unit": "tokens/s", "steps": su["steps"], "ms_per_step": su["total_ms"] / su["steps"],
+            "device_status": su["status"], "clocks": ck,
+            "roofline": roofline(bytes_launch, prefill_flops(w), su["launch_ms"], hbm,
+                                 bf16_sustained, traffic_for(w), peak_src)}
+        if ck and ck.get("sm_mhz"):
+            # the same time at the maximum SM clock, if it scaled with the clock
+            line["sustained"]["ms_per_step_x_mhz_over_max"] = (
+                su["total_ms"] / su["steps"] * ck["sm_mhz"] / ck["sm_max_mhz"])
+    for name, (wx, r) in legs.items():
+        tok = wx.B * wx.N
+        key = {8192: "prefill_8k", 1 << 20: "prefill_1m"}.get(wx.N, wx.name)
+        line[key] = {
+            "workload": wx.name, "value": job_throughput(dist.world, tok, r["total_ms"] / r["steps"]),
+            "unit": "tokens/s", "steps": r["steps"], "ms_per_step": r["total_ms"] / r["steps"],
+            "gpu_launches": r["steps"], "device_status": r["status"],
+            "split": ["whole sequences / chunk scan", "hand-over", "split scan"][
+                ops.fwd_plan(wx.B, wx.H, wx.N, 0, sms)[0]["mode"]],
+            "clocks": sampler.summary([r["window"]]),
+            "roofline": roofline(prefill_bytes(wx), prefill_flops(wx), r["launch_ms"], hbm, bf16,
+                                 traffic_for(wx), peak_src)}
     if dec:
-        gbs = dec["bytes"] / (dec["ms"] / 1e3) / 1e9
-        line["decode"] = {"workload": dec["workload"], "value": dist.world * dec["tokens"] / (dec["ms"] / 1e3),
+        # per head-step: the state read and written (fp32), q, k, v in (bf16),
+        # out (fp32) and the slope; flops: decay, k^T v and q S, 5 D E
+        line["decode"] = {"workload": dec["workload"],
+                          "value": dist.world * dec["tokens"] / (dec["ms"] / 1e3),
                           "unit": "tokens/s", "ms_per_step": dec["ms"], "steps": dec["steps"],
                           "gpu_launches": dec["steps"], "state_finite": dec["finite"],
-                          "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
-                                       "frac": gbs / hbm, "bytes_per_launch": dec["bytes"]}}
+                          "clocks": sampler.summary([dec["window"]]),
+                          "roofline": roofline(dec["bytes"], dec["flops"], dec["ms"], hbm, bf16,
+                                               None, peak_src)}
     if bwd:
         # minimal traffic of the operation: q, k, v, dout read once (bf16), dq,
-        # dk, dv written once (fp32); the three launches move 3 x 1280 B instead
+        # dk, dv written once (fp32); flops: three launches of the blocked form
         units = w.B * w.H * w.N
         bytes_min = units * (2 * (2 * w.D + 2 * w.E) + 4 * (2 * w.D + w.E))
-        bytes_moved = units * (3 * (2 * (w.D + w.D + w.E)) + 4 * (2 * w.D + w.E)) if w.D == w.E \
-            else None
-        gbs = bytes_min / (bwd["ms"] / 1e3) / 1e9
+        r = roofline(bytes_min, 3 * prefill_flops(w), bwd["ms"], hbm, bf16, None, peak_src)
+        r["bytes_moved_by_the_launches"] = bwd["bytes_moved"]
         line["backward"] = {"value": job_throughput(dist.world, tokens_step, bwd["ms"]),
                             "unit": "tokens/s", "ms_per_step": bwd["ms"], "steps": bwd["steps"],
-                            "gpu_launches": 3 * bwd["steps"], "device_status": bwd["status"],
-                            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
-                                         "unit": "GB/s", "frac": gbs / hbm,
-                                         "bytes_per_step": bytes_min,
-                                         "bytes_moved_by_three_launches": bytes_moved}}
+                            "gpu_launches": bwd["launches"] * bwd["steps"],
+                            "device_status": bwd["status"],
+                            "clocks": sampler.summary([bwd["window"]]), "roofline": r}
     if fus:
         # the layer's traffic: raw q, k, v and the gate in (bf16), y out (bf16)
         units = w.B * w.H * w.N
         bytes_layer = units * 2 * (2 * w.D + 3 * w.E)
-        gbs = bytes_layer / (fus["ms"] / 1e3) / 1e9
         line["fused_layer"] = {"value": job_throughput(dist.world, tokens_step, fus["ms"]),
                                "unit": "tokens/s", "ms_per_step": fus["ms"],
                                "steps": fus["steps"], "gpu_launches": fus["steps"],
                                "device_status": fus["status"],
-                               "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
-                                            "unit": "GB/s", "frac": gbs / hbm,
-                                            "bytes_per_step": bytes_layer}}
+                               "clocks": sampler.summary([fus["window"]]),
+                               "roofline": roofline(bytes_layer, prefill_flops(w), fus["ms"], hbm,
+                                                    bf16, None, peak_src)}
     if dist.rank == 0 and dist.world == 1 and args.cpu_seconds > 0:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if dist.rank == 0:

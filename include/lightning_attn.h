@@ -59,7 +59,10 @@ typedef enum {
 } la_status;
 
 /*
- * Prefill, bf16 inputs, fp32 output.
+ * Prefill, bf16 inputs, fp32 output ("MiniMax-M1" model entry, linear/SSM
+ * layer field: the Lightning layer's causal linear attention with a per-head
+ * exponential decay; "MiniMax-01" blog, "What Makes 1M Context Hard": the
+ * linear-complexity variant that carries the long context).
  *   q, k : bf16 [B][H][N][D]      v : bf16 [B][H][N][E]
  *   slopes: fp32 [H], lambda_h    out: fp32 [B][H][N][E] (fully overwritten)
  * Zero initial state.  D, E in {64, 128} (the model's geometry is the
@@ -68,11 +71,20 @@ typedef enum {
  * zero-filled by the tensor maps, which is exact); other D, E return
  * LA_ERR_UNSUPPORTED.  Any N >= 1.
  * Runs on tcgen05 tensor cores (bf16 operands, fp32 accumulation, fp32 state
- * carried on chip).  Work is spread over all SMs: long sequences are split
- * into parts whose entering states come from a state scan or a hand-over;
- * the scratch (at most 2 states of 64 KiB per SM, or per (b, h) with an
- * explicit chunk length) is taken with cudaMallocAsync / cudaFreeAsync on
- * `stream`.
+ * carried on chip).  Work is spread over a persistent grid of one CTA per SM
+ * (capped by lightning_attn_set_cta_limit): long sequences are split into
+ * parts whose entering states come from a state scan or a hand-over; the
+ * scratch (at most 2 states of 64 KiB per CTA, or per (b, h) with an explicit
+ * chunk length) is taken with cudaMallocAsync / cudaFreeAsync on `stream`.
+ * Where CTAs wait for states other CTAs of the same launch publish (the
+ * hand-over when B*H >= CTAs, the split scan when CTAs/8 <= B*H < CTAs), the
+ * launch is cooperative: the runtime starts it only with every CTA resident,
+ * so a kernel running beside it on another stream (or a share of the SMs
+ * held by another process) delays it instead of leaving CTAs waiting for CTAs
+ * that cannot start; if the grid can never be resident the call returns
+ * LA_ERR_CUDA.  The chunk scan (B*H < CTAs/8, or an explicit chunk) hands
+ * work out by ticket in order, so a chunk only waits for a chunk that a
+ * running CTA already holds, and needs no such launch.
  */
 int lightning_attn_fwd(const void* q, const void* k, const void* v,
                        const float* slopes, float* out,
@@ -119,9 +131,12 @@ int lightning_attn_fwd_ex(const void* q, const void* k, const void* v,
  * that would need more than LA_NOALLOC_SCRATCH_BYTES returns LA_ERR_WORKSPACE
  * before launching anything.  With chunk = 0 the split is only used when B*H
  * is below the SM count, which stays within the limit on a 148-SM B200.
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) and caches it; make that first call before any stream
- * capture.  All calls on a device share the one array and it keeps the last
+ * The first call on each device loads the library's device code and looks up
+ * the array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  The address is looked up again on every call
+ * (a host-side table lookup, no allocation), so it stays valid after
+ * cudaDeviceReset re-creates the context.  All calls on a device share the
+ * one array and it keeps the last
  * call's contents (the chunk scan's counters are cleared with cudaMemsetAsync
  * on `stream` at every call; the other splits' flags carry a value unique to
  * the call): calls whose kernels overlap on the GPU -- e.g. issued on
@@ -157,16 +172,24 @@ int lightning_attn_fwd_strided(const void* q, const void* k, const void* v, cons
                                const long long* out_strides, int chunk, void* stream);
 
 /*
- * Prefill with fp32 inputs and output (same operation and layout as
- * lightning_attn_fwd, all tensors fp32).  D, E in {64, 128}.  CUDA-core fp32
- * arithmetic, for callers that need fp32-class accuracy.
+ * Prefill with fp32 inputs and output: the same operation as
+ * lightning_attn_fwd ("MiniMax-M1" model entry, linear/SSM layer field:
+ * causal linear attention with a per-head exponential decay), with the same
+ * layout and all tensors fp32.  D, E in {64, 128}.  CUDA-core fp32 arithmetic,
+ * for callers that need fp32-class accuracy (tensor-core operands would round
+ * to bf16).  One CTA per (b, h) sequence, 32-token blocks, the state in shared
+ * memory; no scratch.  Errors as lightning_attn_fwd.
  */
 int lightning_attn_fwd_f32(const float* q, const float* k, const float* v,
                            const float* slopes, float* out,
                            int B, int H, int N, int D, int E, void* stream);
 
 /*
- * One recurrent decode step for B*H independent (b, h) states.
+ * One recurrent decode step for B*H independent (b, h) states: the Lightning
+ * layer as a fixed-size recurrent state ("MiniMax-M1" model entry, the count
+ * of layers with a fixed-size recurrent state and the linear/SSM layer field's
+ * 128x128 state per head), so a generated token costs one read-modify-write
+ * of the state whatever the context length.
  *   q, k : bf16 [B][H][D]     v : bf16 [B][H][E]
  *   state: fp32 [B][H][D][E] (row d, column e), read and written IN PLACE
  *   out  : fp32 [B][H][E]
@@ -250,6 +273,20 @@ int lightning_attn_fault_test_scan_stall(const void* q, const void* k,
                                          float* out, int B, int H, int N,
                                          int chunk, unsigned int wait_limit_ms,
                                          void* stream);
+
+/*
+ * Caps the persistent grid of every later bf16 prefill-kernel launch of this
+ * process (lightning_attn_fwd, _ex, _strided, _anticausal, _bwd, _fused,
+ * _noalloc) at max_ctas CTAs; 0 removes the cap (one CTA per SM).  For
+ * leaving SMs to other work that runs beside the prefill (a decode step on
+ * another stream, another process); the work splits are planned for the
+ * capped grid, so results do not depend on it beyond rounding.  An interface
+ * for callers, with no counterpart on the pages.  *previous (nullable)
+ * receives the old cap.  Returns LA_ERR_SHAPE for max_ctas < 0.  The setting
+ * is one atomic word shared by all threads; a call that is planning its
+ * launch while another thread changes it uses either value.
+ */
+int lightning_attn_set_cta_limit(int max_ctas, int* previous);
 
 /*
  * Text of the CUDA runtime error behind the calling thread's most recent

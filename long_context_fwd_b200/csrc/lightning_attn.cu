@@ -7,7 +7,6 @@
 
 #include <atomic>
 #include <chrono>
-#include <mutex>
 #include <random>
 
 #include "lightning_attn.h"
@@ -63,6 +62,42 @@ int sm_count() {
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
     return 148;
   return n;
+}
+
+// Caller's cap on the prefill kernel's persistent grid (0 = none), shared by
+// every thread of the process (lightning_attn_set_cta_limit).
+std::atomic<int> g_cta_limit{0};
+
+using FwdKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                           const CUtensorMap, const la::fwd::Params);
+
+FwdKernel pick_fwd_kernel(int rank, bool rev, bool fused) {
+  using la::fwd::fwd_bf16_kernel;
+  return fused       ? fwd_bf16_kernel<3, false, true>
+         : rank == 3 ? (rev ? fwd_bf16_kernel<3, true, false> : fwd_bf16_kernel<3, false, false>)
+                     : (rev ? fwd_bf16_kernel<4, true, false> : fwd_bf16_kernel<4, false, false>);
+}
+
+// Sets the kernel's shared-memory attribute (it belongs to the current
+// device's context, so on every call) and returns in *ctas how many of its
+// CTAs can be resident at once on the current device: SMs x CTAs per SM (one,
+// by design), capped by the caller's limit.  The static work splits plan for
+// exactly that many CTAs and are launched cooperatively, so that either all
+// of them run at the same time or the launch fails up front.
+int prepare_fwd_kernel(FwdKernel kern, int* ctas) {
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::fwd::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, la::fwd::THREADS,
+                                                    la::fwd::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (per_sm < 1) return LA_ERR_UNSUPPORTED;
+  long long n = static_cast<long long>(per_sm) * sm_count();
+  const int cap = g_cta_limit.load(std::memory_order_relaxed);
+  if (cap > 0 && cap < n) n = cap;
+  *ctas = static_cast<int>(n < (1 << 20) ? n : (1 << 20));
+  return LA_OK;
 }
 
 // How the (b, h) sequences become work items for the persistent grid.
@@ -299,19 +334,27 @@ bool build_maps(const void* q, const void* k, const void* v, const void* out, in
   return true;
 }
 
-// Launches the prefill kernel for the map rank (sets the shared-memory
-// attribute on every call: it belongs to the current device's context).
-int launch_fwd(int rank, bool rev, int grid, cudaStream_t stream, const CUtensorMap& tq,
-               const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
-               const la::fwd::Params& p, bool fused = false) {
-  using la::fwd::fwd_bf16_kernel;
-  auto kern = fused     ? fwd_bf16_kernel<3, false, true>
-              : rank == 3 ? (rev ? fwd_bf16_kernel<3, true, false> : fwd_bf16_kernel<3, false, false>)
-                          : (rev ? fwd_bf16_kernel<4, true, false> : fwd_bf16_kernel<4, false, false>);
-  const cudaError_t attr =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::fwd::SMEM_BYTES);
-  if (attr != cudaSuccess) return cuda_fail(attr);
-  kern<<<grid, la::fwd::THREADS, la::fwd::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+// Launches the prefill kernel.  The hand-over and the split scan have CTAs
+// that wait for states other CTAs publish, so those launches are cooperative:
+// the runtime then starts the grid only with every CTA resident (or fails the
+// launch) instead of leaving a waiting CTA on an SM that a CTA it waits for
+// needs.  The chunk scan hands work out by ticket in order and needs no such
+// guarantee.
+int launch_fwd(FwdKernel kern, int grid, bool cooperative, cudaStream_t stream,
+               const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+               const CUtensorMap& to, const la::fwd::Params& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(la::fwd::THREADS);
+  cfg.dynamicSmemBytes = la::fwd::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cooperative ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, p);
+  if (e != cudaSuccess) return cuda_fail(e);
   return launch_status();
 }
 
@@ -343,9 +386,6 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   if (chunk < 0 || (chunk % 128) != 0) return LA_ERR_SHAPE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   const int nseq = B * H;
-  const int sms = sm_count();
-  const Plan pl = make_plan(nseq, N, sms, chunk);
-  if (pl.total >= (1ll << 31)) return LA_ERR_SHAPE;
 
   const Strides st = strides ? *strides : contiguous_strides(H, N, D, E);
   if (!strides_ok(st)) return LA_ERR_ALIGN;
@@ -355,6 +395,12 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   if (!build_maps(q, k, v, out, B, H, N, D, E, st, &tq, &tk, &tv, &to, p, &rank,
                   fused != nullptr))
     return LA_ERR_CUDA;
+  const FwdKernel kern = pick_fwd_kernel(rank, reverse, fused != nullptr);
+  int ctas = 0;
+  int rc = prepare_fwd_kernel(kern, &ctas);
+  if (rc != LA_OK) return rc;
+  const Plan pl = make_plan(nseq, N, ctas, chunk);
+  if (pl.total >= (1ll << 31)) return LA_ERR_SHAPE;
   p.out = fused ? nullptr : static_cast<float*>(out);
   if (fused) {
     p.gate = static_cast<const uint16_t*>(fused->gate);
@@ -390,7 +436,7 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
     set_scratch(pl, scratch, p);
   }
 
-  int rc = launch_fwd(rank, reverse, pl.grid, stream, tq, tk, tv, to, p, fused != nullptr);
+  rc = launch_fwd(kern, pl.grid, pl.mode != la::fwd::MODE_TICKETS, stream, tq, tk, tv, to, p);
   if (scratch) {
     const cudaError_t e = cudaFreeAsync(scratch, stream);
     if (e != cudaSuccess && rc == LA_OK) rc = cuda_fail(e);
@@ -401,28 +447,18 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
 // ---------------------------------------------------------------------------
 // Allocation-free prefill: the chunk-scan scratch lives in a fixed device array.
 // ---------------------------------------------------------------------------
-// The array's name is only a host-side stand-in in host code; its device
-// address is fetched per device with cudaGetSymbolAddress (first call on each
-// device) and cached.
+// In host code the array's name is only a host-side stand-in: its device
+// address in the current device's context is looked up with
+// cudaGetSymbolAddress on every call (a table lookup once the library's device
+// code is loaded, which the first call on each device does), so a context that
+// was reset and re-created never gets a stale address.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
 int noalloc_scratch_ptr(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (dev < 0 || dev >= kMaxDevices) return LA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_fail(e);
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
+  *out = ptr;
   return LA_OK;
 }
 
@@ -437,7 +473,14 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
   if (chunk < 0 || (chunk % 128) != 0) return LA_ERR_SHAPE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
   const int nseq = B * H;
-  const int sms = sm_count();
+  // an explicit chunk length's scratch (two states per sequence) does not
+  // depend on the grid: rejected on the host before touching the device
+  if (chunk > 0 && make_plan(nseq, N, 1, chunk).bytes > LA_NOALLOC_SCRATCH_BYTES)
+    return LA_ERR_WORKSPACE;
+  const FwdKernel kern = pick_fwd_kernel(3, false, false);
+  int sms = 0;
+  const int prc = prepare_fwd_kernel(kern, &sms);
+  if (prc != LA_OK) return prc;
   Plan pl = make_plan(nseq, N, sms, chunk);
   if (pl.mode != la::fwd::MODE_TICKETS && pl.bytes > LA_NOALLOC_SCRATCH_BYTES) {
     // a GPU with so many SMs that the chunk states do not fit: whole sequences
@@ -480,7 +523,7 @@ int fwd_bf16_noalloc_impl(const void* q, const void* k, const void* v, const flo
     }
     set_scratch(pl, scratch, p);
   }
-  return launch_fwd(rank, false, pl.grid, stream, tq, tk, tv, to, p);
+  return launch_fwd(kern, pl.grid, pl.mode != la::fwd::MODE_TICKETS, stream, tq, tk, tv, to, p);
 }
 
 template <int D, int E>
@@ -612,6 +655,13 @@ int lightning_attn_decode(const void* q, const void* k, const void* v, float* st
 }
 
 const char* lightning_attn_last_cuda_error(void) { return t_last_cuda_error; }
+
+int lightning_attn_set_cta_limit(int max_ctas, int* previous) {
+  if (max_ctas < 0) return LA_ERR_SHAPE;
+  const int old = g_cta_limit.exchange(max_ctas);
+  if (previous) *previous = old;
+  return LA_OK;
+}
 
 int lightning_attn_fwd_plan(int B, int H, int N, int chunk, int sms, int* info, int* rec,
                             int max_rec, int* n_rec) {

@@ -43,6 +43,7 @@ SIGNATURES = {
     "lightning_attn_bwd": [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P],
     "lightning_attn_fwd_strided": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P,
                                    _I, _P],
+    "lightning_attn_set_cta_limit": [_I, _P],
 }
 
 
@@ -351,6 +352,15 @@ def fault_test_scan_stall(q, k, v, slopes, out, *, chunk: int, wait_limit_ms: in
         q.data_ptr(), k.data_ptr(), v.data_ptr(), slopes.data_ptr(), out.data_ptr(), B, H, N,
         int(chunk), int(wait_limit_ms), _stream_handle(stream))
     _check("lightning_attn_fault_test_scan_stall", rc)
+
+
+def set_cta_limit(max_ctas: int) -> int:
+    """Caps the prefill kernel's persistent grid for later calls (0 = one CTA
+    per SM); returns the previous cap.  Process-wide."""
+    prev = ctypes.c_int(0)
+    _check("lightning_attn_set_cta_limit",
+           lib().lightning_attn_set_cta_limit(int(max_ctas), ctypes.byref(prev)))
+    return prev.value
 
 
 def device_status(reset: bool = True) -> int:

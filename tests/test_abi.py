@@ -164,3 +164,16 @@ def test_fused_layer_validation(lib):
     assert f(*ok[:6], -1.0, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_SHAPE
     assert f(*ok[:6], float("nan"), FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_SHAPE
     assert f(*ok[:6], 1e-6, FAKE, 1, 1, 8, 128, 96, None) == LA_ERR_UNSUPPORTED
+
+
+def test_cta_limit_setter(lib):
+    prev = ops.set_cta_limit(0)
+    try:
+        assert ops.set_cta_limit(17) == 0
+        assert ops.set_cta_limit(0) == 17
+        with pytest.raises(ops.LightningAttnError) as err:
+            ops.set_cta_limit(-1)
+        assert err.value.code == LA_ERR_SHAPE
+        assert ops.set_cta_limit(0) == 0  # a rejected call leaves the cap alone
+    finally:
+        ops.set_cta_limit(prev)

@@ -32,11 +32,12 @@ def test_decode_geometries_chain(D, E):
 def test_decode_workload_1024_steps_sampled_rows():
     """256 sequences x 64 heads, 1024 chained steps from N(0, 0.02^2) states.
 
-    All rows run on the GPU; three batch rows (192 heads) are drawn on the host
-    and followed step by step by the oracle.
+    All rows run on the GPU; sixteen batch rows (1024 heads, spread over the
+    batch) are drawn on the host and followed step by step by the oracle.
     """
     w = I.DECODE
-    rows = [0, 101, 255]
+    rows = list(range(0, 256, 17))
+    assert len(rows) == 16 and rows[-1] == 255
     s0 = I.decode_state(w)
     sl = I.slopes_for(w)
     state = f32_to_dev(s0, DEV)

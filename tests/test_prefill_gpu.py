@@ -10,7 +10,8 @@ import torch
 import oracle
 from long_context_fwd_b200 import inputs as I
 from long_context_fwd_b200 import ops
-from parity import TOL_BF16, TOL_F32, bf16_to_dev, f32_to_dev, rel, worst_head
+from parity import (TOL_BF16, TOL_F32, bf16_to_dev, f32_to_dev, fill_heads_from_host,
+                    host_workers, rel, worst_head)
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -284,56 +285,67 @@ def test_bf16_prefill_8k_workload_full():
     assert worst_head(got, ref) <= TOL_BF16
 
 
-def _device_workload_with_host_heads(w, heads):
-    """Full-size inputs on the device (torch generator) with the listed heads
-    replaced by the host generator's draws, which the oracle also consumes."""
-    q, k, v = I.device_prefill_inputs(w, DEV)
-    host = {}
-    for b, h in heads:
-        hq, hk, hv = I.head_inputs(w, b, h)
-        q[b, h].copy_(bf16_to_dev(hq, DEV))
-        k[b, h].copy_(bf16_to_dev(hk, DEV))
-        v[b, h].copy_(bf16_to_dev(hv, DEV))
-        host[(b, h)] = (hq, hk, hv)
-    return q, k, v, host
-
-
-def test_bf16_prefill_32k_workload_sampled_heads():
+def test_bf16_prefill_32k_workload_every_sequence():
     """B=4, H=64, N=32768 (lambda = 0 on heads h % 8 == 7), as the benchmark runs
-    it; eight heads (three with lambda = 0) compared in full against the oracle."""
+    it, every (b, h) input drawn on the host: all 256 sequences checked at the
+    64 sampled positions, and 48 of them -- all 32 lambda = 0 heads and 16
+    decaying ones -- in full, against the oracle's recurrence."""
     w = I.PREFILL_32K
-    heads = [(0, 0), (0, 7), (1, 31), (1, 63), (2, 15), (2, 40), (3, 1), (3, 55)]
     sl = I.slopes_for(w)
-    q, k, v, host = _device_workload_with_host_heads(w, heads)
+    pos = I.sample_positions(w.N)
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    full = {(b, h) for b, h in heads if sl[h] == 0.0 or h in (0, 20, 41, 62)}
+    assert len(full) == 48 and sum(sl[h] == 0.0 for _, h in full) == 32
+    q, k, v = (torch.empty((w.B, w.H, w.N, 128), dtype=torch.bfloat16, device=DEV)
+               for _ in range(3))
+
+    def reference(b, h, hq, hk, hv):
+        args = (hq[None, None], hk[None, None], hv[None, None], sl[h:h + 1])
+        if (b, h) in full:
+            return oracle.recurrent(*args, threads=1)[0, 0]
+        return oracle.recurrent_sampled(*args, pos, threads=1)[0, 0]
+
+    refs = fill_heads_from_host(lambda b, h: I.head_inputs(w, b, h), (q, k, v), heads, reference,
+                                host_workers(0.4e9))
     out = ops.fwd(q, k, v, f32_to_dev(sl, DEV))
     torch.cuda.synchronize()
     assert ops.device_status(reset=True) == 0
     del q, k, v
-    for (b, h), (hq, hk, hv) in host.items():
-        ref = oracle.recurrent(hq[None, None], hk[None, None], hv[None, None], sl[h:h + 1])
-        got = out[b, h].cpu().numpy()
-        assert rel(got, ref[0, 0]) <= TOL_BF16, (b, h)
+    idx = torch.as_tensor(pos, device=DEV)
+    sampled = out.index_select(2, idx).cpu().numpy()  # [B, H, 64, E]
+    for (b, h), ref in refs.items():
+        if (b, h) in full:
+            got = out[b, h].cpu().numpy()
+            assert rel(got, ref) <= TOL_BF16, (b, h)
+            ref = ref[pos]
+        assert rel(sampled[b, h], ref) <= TOL_BF16, (b, h)
+    at_pos = lambda b, h: refs[(b, h)][pos] if (b, h) in full else refs[(b, h)]
+    ref_all = np.stack([np.stack([at_pos(b, h) for h in range(w.H)]) for b in range(w.B)])
+    assert rel(sampled, ref_all) <= TOL_BF16
     assert torch.isfinite(out).all()
 
 
 @pytest.mark.slow
-def test_bf16_prefill_1m_workload_sampled():
-    """B=1, H=64, N=1,048,576: three heads checked at 64 sampled positions each
-    against the oracle's recurrence."""
+def test_bf16_prefill_1m_workload_every_head_sampled():
+    """B=1, H=64, N=1,048,576, as the benchmark runs it, every head's inputs drawn
+    on the host: each of the 64 heads checked at the 64 sampled positions against
+    the oracle's recurrence over all 1,048,576 tokens."""
     w = I.PREFILL_1M
-    heads = [(0, 0), (0, 31), (0, 63)]
     sl = I.slopes_for(w)
-    q, k, v, host = _device_workload_with_host_heads(w, heads)
+    pos = I.sample_positions(w.N)
+    q, k, v = (torch.empty((w.B, w.H, w.N, 128), dtype=torch.bfloat16, device=DEV)
+               for _ in range(3))
+    refs = fill_heads_from_host(
+        lambda b, h: I.head_inputs(w, b, h), (q, k, v), [(0, h) for h in range(w.H)],
+        lambda b, h, hq, hk, hv: oracle.recurrent_sampled(
+            hq[None, None], hk[None, None], hv[None, None], sl[h:h + 1], pos, threads=1)[0, 0],
+        host_workers(2.5e9))
     out = ops.fwd(q, k, v, f32_to_dev(sl, DEV))
     torch.cuda.synchronize()
     assert ops.device_status(reset=True) == 0
     del q, k, v
-    pos = I.sample_positions(w.N)
-    hq = np.stack([host[x][0] for x in heads])[None]
-    hk = np.stack([host[x][1] for x in heads])[None]
-    hv = np.stack([host[x][2] for x in heads])[None]
-    ref = oracle.recurrent_sampled(hq, hk, hv, sl[[h for _, h in heads]], pos)
-    idx = torch.as_tensor(pos, device=DEV)
-    for i, (b, h) in enumerate(heads):
-        got = out[b, h].index_select(0, idx).cpu().numpy()
-        assert rel(got, ref[0, i]) <= TOL_BF16, (b, h)
+    got = out[0].index_select(1, torch.as_tensor(pos, device=DEV)).cpu().numpy()  # [H, 64, E]
+    ref = np.stack([refs[(0, h)] for h in range(w.H)])
+    for h in range(w.H):
+        assert rel(got[h], ref[h]) <= TOL_BF16, h
+    assert rel(got, ref) <= TOL_BF16

@@ -7,16 +7,18 @@ fail).  It keeps the chunk-scan scratch in one fixed device array compiled
 into the library instead of calling cudaMallocAsync.  This test calls it
 through the C ABI twice in a row on different inputs -- the second call reuses
 the array the first one left behind -- and checks each result against the
-allocating entry point on the same inputs, with the bf16 tolerance used by the
-other prefill tests.  The file is named so that pytest collects it last.
+allocating entry point on the same inputs and against the float64 oracle, with
+the bf16 tolerance used by the other prefill tests.  The file is named so that
+pytest collects it last.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from long_context_fwd_b200 import inputs as I
 from long_context_fwd_b200 import ops
-from parity import TOL_BF16, bf16_to_dev, f32_to_dev, rel
+from parity import TOL_BF16, bf16_to_dev, f32_to_dev, rel, worst_head
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -25,8 +27,9 @@ DEV = torch.device("cuda:0")
 def _case(seed, B, H, N, slopes):
     w = I.Workload(f"noalloc{seed}", B, H, N, 128, 128, "bf16", index=400 + seed)
     q, k, v = I.prefill_inputs(w)
-    return (bf16_to_dev(q, DEV), bf16_to_dev(k, DEV), bf16_to_dev(v, DEV),
-            f32_to_dev(np.asarray(slopes, np.float32), DEV))
+    sl = np.asarray(slopes, np.float32)
+    return (bf16_to_dev(q, DEV), bf16_to_dev(k, DEV), bf16_to_dev(v, DEV), f32_to_dev(sl, DEV),
+            oracle.recurrent(q, k, v, sl))
 
 
 @pytest.mark.parametrize("chunk", [0, 256])
@@ -38,7 +41,7 @@ def test_noalloc_matches_allocating_entry_point_twice(chunk):
         # more sequences than SMs: the balanced split hands sequences over
         # between CTAs through the same fixed array
         cases.append(_case(3, 1, 150, 1100, [0.5, 0.02, 0.0] * 50))
-    for q, k, v, sl in cases:
+    for q, k, v, sl, want in cases:
         out_na = torch.full(q.shape[:3] + (128,), float("nan"), dtype=torch.float32, device=DEV)
         ops.fwd_noalloc(q, k, v, sl, out_na, chunk=chunk)
         ref = ops.fwd(q, k, v, sl, chunk=chunk)
@@ -47,6 +50,8 @@ def test_noalloc_matches_allocating_entry_point_twice(chunk):
         a, b = out_na.cpu().numpy(), ref.cpu().numpy()
         assert np.isfinite(a).all()
         assert rel(a, b) <= TOL_BF16
+        assert rel(a, want) <= TOL_BF16
+        assert worst_head(a, want) <= TOL_BF16
 
 
 def test_noalloc_rejects_scratch_beyond_limit():
