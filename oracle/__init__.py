@@ -73,8 +73,8 @@ def _load():
                                                       I64, I64, I]
             lib.la_oracle_backward_recurrent.argtypes = [P, P, P, P, I, P, P, P, P, I64, I64, I64,
                                                          I64, I64, I]
-            lib.la_oracle_fused_layer.argtypes = [P, P, P, P, I, P, P, ctypes.c_double, P, I64,
-                                                  I64, I64, I64, I64, I]
+            lib.la_oracle_fused_layer.argtypes = [P, P, P, P, I, P, P, ctypes.c_double, P, P, P,
+                                                  I64, I64, I64, I64, I64, I]
             for f in ("la_oracle_masked", "la_oracle_recurrent", "la_oracle_recurrent_sampled",
                       "la_oracle_blocked", "la_oracle_decode_step", "la_oracle_max_threads",
                       "la_oracle_masked_anticausal", "la_oracle_recurrent_anticausal",
@@ -230,11 +230,14 @@ def backward(q, k, v, dout, slopes, form: str = "recurrent", threads: int = 0):
     return dq, dk, dv
 
 
-def fused_layer(q, k, v, gate, slopes, norm_weight, eps: float, threads: int = 0) -> np.ndarray:
+def fused_layer(q, k, v, gate, slopes, norm_weight, eps: float, s0=None,
+                return_state: bool = False, threads: int = 0):
     """The layer around the operator, float64 [B,H,N,E]:
     y = w * RMSNorm_E(o) * sigmoid(gate) with o the recurrence on (silu(q),
     silu(k), silu(v)); the RMSNorm runs over each head's E outputs and w is
-    per channel, norm_weight [H, E] (or [H * E])."""
+    per channel, norm_weight [H, E] (or [H * E]).  s0: optional initial state
+    [B,H,D,E] of the recurrence (on the activated k, v); with return_state the
+    state after the last token is returned too: (y, state)."""
     q, k, v, dt = _inputs(q, k, v)
     g = np.ascontiguousarray(gate)
     if g.dtype != q.dtype:
@@ -248,10 +251,13 @@ def fused_layer(q, k, v, gate, slopes, norm_weight, eps: float, threads: int = 0
         raise ValueError("norm_weight must have H * E entries")
     s = _slopes(slopes, H)
     out = np.empty((B, H, N, E), dtype=np.float64)
+    s0a = None if s0 is None else np.ascontiguousarray(s0, dtype=np.float64).reshape(B, H, D, E)
+    sf = np.empty((B, H, D, E), dtype=np.float64) if return_state else None
     _check(_load().la_oracle_fused_layer(_ptr(q), _ptr(k), _ptr(v), _ptr(g), dt, _ptr(s),
-                                         _ptr(w), float(eps), _ptr(out), B, H, N, D, E, threads),
+                                         _ptr(w), float(eps), _ptr(s0a), _ptr(sf), _ptr(out),
+                                         B, H, N, D, E, threads),
            "la_oracle_fused_layer")
-    return out
+    return (out, sf) if return_state else out
 
 
 def max_threads() -> int:

@@ -52,6 +52,11 @@
  *        (silu(q), silu(k), silu(v)), RMSNorm over each head's E outputs:
  *        RMSNorm(o_t) = o_t / sqrt(mean_e(o_te^2) + eps); w per channel
  *        (h * E + e); silu(x) = x / (1 + exp(-x)); sigmoid(x) = 1/(1+exp(-x)).
+ *        Optionally from an initial state S_0 (nullable, [B][H][D][E]) and
+ *        returning the state after the last token (nullable): the layer's
+ *        fixed-size recurrent state (same entry, the count of layers with a
+ *        fixed-size recurrent state), so that a sequence can continue token by
+ *        token (N = 1 is one decode step of the layer).
  */
 #include <math.h>
 #include <stdint.h>
@@ -516,8 +521,9 @@ static double silu(double x) { return x / (1.0 + exp(-x)); }
 static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 
 int la_oracle_fused_layer(const void* q, const void* k, const void* v, const void* gate, int dtype,
-                          const float* slopes, const float* norm_w, double eps, double* out,
-                          int64_t B, int64_t H, int64_t N, int64_t D, int64_t E, int nthreads) {
+                          const float* slopes, const float* norm_w, double eps, const double* s0,
+                          double* sf, double* out, int64_t B, int64_t H, int64_t N, int64_t D,
+                          int64_t E, int nthreads) {
   int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
   if (rc) return rc;
   if (!gate || !norm_w || !(eps >= 0.0)) return 1;
@@ -533,6 +539,7 @@ int la_oracle_fused_layer(const void* q, const void* k, const void* v, const voi
     double* vt = (double*)malloc(sizeof(double) * (size_t)E);
     double* ot = (double*)malloc(sizeof(double) * (size_t)E);
     double* Y = out + bh * N * E;
+    if (s0) memcpy(S, s0 + bh * D * E, sizeof(double) * (size_t)(D * E));
     for (int64_t t = 0; t < N; ++t) {
       in_row(qt, q, (bh * N + t) * D, D, dtype);
       in_row(kt, k, (bh * N + t) * D, D, dtype);
@@ -557,6 +564,7 @@ int la_oracle_fused_layer(const void* q, const void* k, const void* v, const voi
         Y[t * E + e] = (double)norm_w[h * E + e] * ot[e] * rinv * sigmoid(g);
       }
     }
+    if (sf) memcpy(sf + bh * D * E, S, sizeof(double) * (size_t)(D * E));
     free(S);
     free(qt);
     free(kt);

@@ -127,3 +127,69 @@ def test_layer_rejects_bad_arguments():
         oracle.fused_layer(q, q, q, q.astype(np.float64), [0.1], np.ones(2), 1e-6)
     with pytest.raises(ValueError):
         oracle.fused_layer(q, q, q, q, [0.1], np.ones(2), -1.0)
+
+
+def _python_layer_state(q, k, v, g, lam, w, eps, s0):
+    """Pure Python, from an initial state S_0 (D x E): the operator's output gains
+    gamma^(t+1) silu(q_t) S_0, and the final state is
+    gamma^N S_0 + sum_s gamma^(N-1-s) silu(k_s)^T silu(v_s)."""
+    silu = lambda x: x / (1.0 + math.exp(-x))
+    N, D, E = len(q), len(q[0]), len(v[0])
+    gam = math.exp(-lam)
+    qs = [[silu(float(x)) for x in row] for row in q]
+    ks = [[silu(float(x)) for x in row] for row in k]
+    vs = [[silu(float(x)) for x in row] for row in v]
+    o = brute_force(qs, ks, vs, lam)
+    y = []
+    for t in range(N):
+        row = [o[t][e] + gam ** (t + 1) * sum(qs[t][d] * float(s0[d][e]) for d in range(D))
+               for e in range(E)]
+        r = 1.0 / math.sqrt(sum(x * x for x in row) / E + eps)
+        y.append([float(w[e]) * row[e] * r / (1.0 + math.exp(-float(g[t][e]))) for e in range(E)])
+    sf = [[gam ** N * float(s0[d][e]) +
+           sum(gam ** (N - 1 - s) * ks[s][d] * vs[s][e] for s in range(N))
+           for e in range(E)] for d in range(D)]
+    return y, sf
+
+
+@pytest.mark.parametrize("N,D,E,lam", [(1, 3, 4, 0.3), (11, 4, 3, 0.0), (6, 2, 5, 1.7)])
+def test_layer_state_in_and_out_match_python_statement(N, D, E, lam):
+    H = 2
+    q, k, v = _rand((1, H, N, D), 21), _rand((1, H, N, D), 22), _rand((1, H, N, E), 23)
+    g = _rand((1, H, N, E), 24, 2.0)
+    w = _rand((H, E), 25) + 1.0
+    s0 = _rand((1, H, D, E), 26, 0.5).astype(np.float64)
+    sl = [lam, 0.4]
+    y, sf = oracle.fused_layer(q, k, v, g, sl, w, 1e-6, s0=s0, return_state=True)
+    for h in range(H):
+        ry, rs = _python_layer_state(q[0, h], k[0, h], v[0, h], g[0, h],
+                                     float(np.float32(sl[h])), w[h], 1e-6, s0[0, h])
+        assert _rel(y[0, h], np.array(ry)) <= 1e-12
+        assert _rel(sf[0, h], np.array(rs)) <= 1e-12
+
+
+def test_layer_continues_a_sequence_from_its_state():
+    # the layer over N tokens equals the layer over the first N1 tokens followed
+    # by the layer over the rest started from the state the first part returned;
+    # the last N - N2 tokens one at a time (decode steps of the layer) too
+    B, H, N, N1, N2, D, E = 2, 3, 40, 17, 35, 6, 5
+    q, k, v = _rand((B, H, N, D), 31), _rand((B, H, N, D), 32), _rand((B, H, N, E), 33)
+    g = _rand((B, H, N, E), 34, 2.0)
+    w = _rand((H, E), 35) + 1.0
+    sl = [0.0, 0.2, 1.3]
+    full, sfull = oracle.fused_layer(q, k, v, g, sl, w, 1e-6, return_state=True)
+    a, sa = oracle.fused_layer(q[:, :, :N1], k[:, :, :N1], v[:, :, :N1], g[:, :, :N1], sl, w,
+                               1e-6, return_state=True)
+    b, sb = oracle.fused_layer(q[:, :, N1:N2], k[:, :, N1:N2], v[:, :, N1:N2], g[:, :, N1:N2],
+                               sl, w, 1e-6, s0=sa, return_state=True)
+    parts = [a, b]
+    s = sb
+    for t in range(N2, N):
+        y, s = oracle.fused_layer(q[:, :, t:t + 1], k[:, :, t:t + 1], v[:, :, t:t + 1],
+                                  g[:, :, t:t + 1], sl, w, 1e-6, s0=s, return_state=True)
+        parts.append(y)
+    assert _rel(np.concatenate(parts, axis=2), full) <= 1e-13
+    assert _rel(s, sfull) <= 1e-13
+    # a zero initial state is the same as none
+    np.testing.assert_array_equal(
+        oracle.fused_layer(q, k, v, g, sl, w, 1e-6, s0=np.zeros((B, H, D, E))), full)
