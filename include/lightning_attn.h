@@ -250,11 +250,68 @@ int lightning_attn_bwd(const void* q, const void* k, const void* v, const void* 
  * sigmoids), the norm, weight and gate in the epilogue, which stores bf16:
  * 256 B of output per token-head instead of 512.  Zero initial state; D, E in
  * {64, 128}; contiguous tensors, 16-byte aligned (else LA_ERR_ALIGN); errors
- * otherwise as lightning_attn_fwd.
+ * otherwise as lightning_attn_fwd.  lightning_attn_fwd_fused_ex adds strides
+ * and the state in and out.
  */
 int lightning_attn_fwd_fused(const void* q, const void* k, const void* v, const void* gate,
                              const float* slopes, const float* norm_weight, float eps, void* out,
                              int B, int H, int N, int D, int E, void* stream);
+
+/*
+ * The fused layer (as lightning_attn_fwd_fused) for a model's layer: inputs
+ * read in the layouts a QKV projection writes, and the recurrent state handed
+ * in and out so a sequence can be prefilled in pieces and then continued token
+ * by token with lightning_attn_decode_fused ("MiniMax-M1" model entry:
+ * linear-layer field -- SiLU on Q, K, V, RMSNorm on the output, 128x128 state
+ * per head; gate field -- sigmoid gate after the RMSNorm; the count of layers
+ * with a fixed-size recurrent state).
+ *   init_state : nullable fp32 [B][H][D][E], the state before token 0 of the
+ *                recurrence on the activated k, v (zero if NULL)
+ *   final_state: nullable fp32 [B][H][D][E], receives the state after token N-1
+ *   q_strides, k_strides, v_strides, gate_strides, out_strides: {b, h, t}
+ *                element strides of each tensor (the last dimension
+ *                contiguous), all five NULL for contiguous head-major
+ *                [B][H][N][*] tensors, else all five non-NULL (LA_ERR_NULL
+ *                otherwise).  E.g. token-major [B][N][H][*] is {N*H*W, W,
+ *                H*W}; slices of one fused [B][N][3][H][D] projection output
+ *                {3*N*H*D, D, 3*H*D}.  Every stride times 2 bytes a multiple of
+ *                16 below 2^40, every pointer 16-byte aligned (LA_ERR_ALIGN).
+ *   chunk      : as lightning_attn_fwd_ex.
+ * Everything else -- the computation, eps, norm_weight [H][E], bf16 out,
+ * D, E in {64, 128}, the errors -- as lightning_attn_fwd_fused.
+ */
+int lightning_attn_fwd_fused_ex(const void* q, const void* k, const void* v, const void* gate,
+                                const float* slopes, const float* norm_weight, float eps,
+                                const float* init_state, float* final_state, void* out, int B,
+                                int H, int N, int D, int E, const long long* q_strides,
+                                const long long* k_strides, const long long* v_strides,
+                                const long long* gate_strides, const long long* out_strides,
+                                int chunk, void* stream);
+
+/*
+ * One decode step of the fused layer: the layer's fixed-size recurrent state
+ * advanced by one token ("MiniMax-M1" model entry, the count of layers with a
+ * fixed-size recurrent state; linear-layer field: SiLU on Q, K, V, RMSNorm on
+ * the output; gate field: sigmoid gate after the RMSNorm), per (b, h):
+ *   state <- exp(-lambda_h) state + silu(k)^T silu(v);   o = silu(q) . state
+ *   out    = norm_weight[h] * o / sqrt(mean_e(o_e^2) + eps) * sigmoid(gate)
+ *   q, k : bf16 [B][H][D], raw projections     v, gate : bf16 [B][H][E], raw
+ *   state: fp32 [B][H][D][E], contiguous, updated IN PLACE (the final_state of
+ *          lightning_attn_fwd_fused_ex continues here)
+ *   norm_weight: fp32 [H][E]   eps: finite, >= 0 (else LA_ERR_SHAPE)
+ *   out  : bf16 [B][H][E]
+ *   *_strides: {b, h} element strides of q, k, v, gate and out, all five NULL
+ *          for the contiguous layouts above, else all five non-NULL; each a
+ *          non-negative multiple of 8 elements below 2^40 (LA_ERR_ALIGN).
+ * D, E in {64, 128}; every pointer 16-byte aligned except slopes and
+ * norm_weight (4).  One CTA per (b, h); HBM-bound like lightning_attn_decode.
+ */
+int lightning_attn_decode_fused(const void* q, const void* k, const void* v, const void* gate,
+                                float* state, const float* slopes, const float* norm_weight,
+                                float eps, void* out, int B, int H, int D, int E,
+                                const long long* q_strides, const long long* k_strides,
+                                const long long* v_strides, const long long* gate_strides,
+                                const long long* out_strides, void* stream);
 
 /*
  * Fault-injection hook for testing the bounded device-side waits (an interface

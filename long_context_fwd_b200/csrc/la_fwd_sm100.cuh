@@ -1017,8 +1017,10 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         // its outputs will take, while the row's mean square is computed; each
         // output chunk then overwrites its own gate chunk.
         const int tok = row + static_cast<int>(r);
-        const uint16_t* grow =
-            tok < p.N ? p.gate + (static_cast<int64_t>(it.seq) * p.N + tok) * p.E : nullptr;
+        const uint16_t* grow = tok < p.N ? p.gate + (it.seq / p.H) * p.gstride[0] +
+                                               (it.seq % p.H) * p.gstride[1] +
+                                               static_cast<int64_t>(tok) * p.gstride[2]
+                                         : nullptr;
         const uint32_t srow = vtile + r * 128u;
         if (grow) {
 #pragma unroll

@@ -39,7 +39,8 @@ struct Params {
                               // the tensor maps zero-fill the columns past D or E)
   float* out;                 // the output and its element strides {b, h, t}, for rows that
   long long ostride[3];       // are stored without TMA (anti-causal runs, first block)
-  const uint16_t* gate;       // fused layer: bf16 gate [B][H][N][E] (before the sigmoid)
+  const uint16_t* gate;       // fused layer: bf16 gate (before the sigmoid), element
+  long long gstride[3];       // strides {b, h, t}, e contiguous
   const float* norm_w;        // fused layer: RMSNorm weight [H][E]
   float eps;                  // fused layer: RMSNorm epsilon
   unsigned long long wait_limit_ns;

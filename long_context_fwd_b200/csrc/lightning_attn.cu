@@ -73,9 +73,9 @@ using FwdKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorM
 
 FwdKernel pick_fwd_kernel(int rank, bool rev, bool fused) {
   using la::fwd::fwd_bf16_kernel;
-  return fused       ? fwd_bf16_kernel<3, false, true>
-         : rank == 3 ? (rev ? fwd_bf16_kernel<3, true, false> : fwd_bf16_kernel<3, false, false>)
-                     : (rev ? fwd_bf16_kernel<4, true, false> : fwd_bf16_kernel<4, false, false>);
+  if (fused) return rank == 3 ? fwd_bf16_kernel<3, false, true> : fwd_bf16_kernel<4, false, true>;
+  return rank == 3 ? (rev ? fwd_bf16_kernel<3, true, false> : fwd_bf16_kernel<3, false, false>)
+                   : (rev ? fwd_bf16_kernel<4, true, false> : fwd_bf16_kernel<4, false, false>);
 }
 
 // Sets the kernel's shared-memory attribute (it belongs to the current
@@ -261,15 +261,16 @@ unsigned long long launch_tag() {
   }
 }
 
-// Element strides {b, h, t} of q, k, v and out (d or e contiguous).
+// Element strides {b, h, t} of q, k, v, out and the fused layer's gate (d or e
+// contiguous).
 struct Strides {
-  long long s[4][3];
+  long long s[5][3];
 };
 
 Strides contiguous_strides(int H, int N, int D, int E) {
   Strides st;
-  const long long w[4] = {D, D, E, E};
-  for (int i = 0; i < 4; ++i) {
+  const long long w[5] = {D, D, E, E, E};
+  for (int i = 0; i < 5; ++i) {
     st.s[i][2] = w[i];
     st.s[i][1] = static_cast<long long>(N) * w[i];
     st.s[i][0] = static_cast<long long>(H) * N * w[i];
@@ -277,10 +278,11 @@ Strides contiguous_strides(int H, int N, int D, int E) {
   return st;
 }
 
-// TMA needs every stride in bytes to be a multiple of 16 and below 2^40.
-bool strides_ok(const Strides& st) {
-  const int eb[4] = {2, 2, 2, 4};
-  for (int i = 0; i < 4; ++i)
+// TMA needs every stride in bytes to be a multiple of 16 and below 2^40 (the
+// gate's rows are read with 16-byte copies, which need the same).
+bool strides_ok(const Strides& st, bool out_bf16) {
+  const int eb[5] = {2, 2, 2, out_bf16 ? 2 : 4, 2};
+  for (int i = 0; i < 5; ++i)
     for (int j = 0; j < 3; ++j) {
       const long long b = st.s[i][j] * eb[i];
       if (st.s[i][j] < 0 || b % 16 != 0 || b >= (1ll << 40)) return false;
@@ -302,7 +304,7 @@ bool build_maps(const void* q, const void* k, const void* v, const void* out, in
   p.E = E;
   const Strides cont = contiguous_strides(H, N, D, E);
   bool contiguous = true;
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 4; ++i)  // q, k, v, out (the gate is read without a map)
     for (int j = 0; j < 3; ++j) {
       const bool unused = (j == 0 && B == 1) || (j == 1 && H == 1);  // extent-1 dimension
       contiguous = contiguous && (unused || st.s[i][j] == cont.s[i][j]);
@@ -317,7 +319,6 @@ bool build_maps(const void* q, const void* k, const void* v, const void* out, in
                      : la::make_tmap_3d(to, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, E, N, nseq, 32, 128));
   }
   *rank = 4;
-  if (out_bf16) return false;  // the fused layer takes contiguous tensors only
   const uint64_t ext[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(H),
                            static_cast<uint64_t>(B)};
   CUtensorMap* maps[4] = {tq, tk, tv, to};
@@ -325,7 +326,7 @@ bool build_maps(const void* q, const void* k, const void* v, const void* out, in
   for (int i = 0; i < 4; ++i) {
     const uint64_t str[3] = {static_cast<uint64_t>(st.s[i][2]), static_cast<uint64_t>(st.s[i][1]),
                              static_cast<uint64_t>(st.s[i][0])};
-    const bool f32 = i == 3;
+    const bool f32 = i == 3 && !out_bf16;
     if (!la::make_tmap_4d(maps[i], bases[i],
                           f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                           f32 ? 4 : 2, i < 2 ? D : E, ext, str, f32 ? 32 : 64, 128, &p.cslot[i]))
@@ -376,7 +377,7 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
     if (!fused->gate || !fused->norm_w) return LA_ERR_NULL;
     if (!aligned16(fused->gate) || !aligned16(fused->norm_w)) return LA_ERR_ALIGN;
     if (!(fused->eps >= 0.f) || fused->eps > 3.0e38f) return LA_ERR_SHAPE;
-    if (strides || reverse) return LA_ERR_UNSUPPORTED;
+    if (reverse) return LA_ERR_UNSUPPORTED;
   }
   if (!dims_ok(B, H, N, D, E)) return LA_ERR_SHAPE;
   if ((D != 64 && D != 128) || (E != 64 && E != 128)) return LA_ERR_UNSUPPORTED;
@@ -388,7 +389,7 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
   const int nseq = B * H;
 
   const Strides st = strides ? *strides : contiguous_strides(H, N, D, E);
-  if (!strides_ok(st)) return LA_ERR_ALIGN;
+  if (!strides_ok(st, fused != nullptr)) return LA_ERR_ALIGN;
   la::fwd::Params p{};
   CUtensorMap tq, tk, tv, to;
   int rank = 3;
@@ -406,6 +407,7 @@ int fwd_bf16_impl(const void* q, const void* k, const void* v, const float* slop
     p.gate = static_cast<const uint16_t*>(fused->gate);
     p.norm_w = fused->norm_w;
     p.eps = fused->eps;
+    for (int j = 0; j < 3; ++j) p.gstride[j] = st.s[4][j];
   }
   for (int j = 0; j < 3; ++j) p.ostride[j] = st.s[3][j];
 
@@ -547,6 +549,12 @@ int launch_decode(const void* q, const void* k, const void* v, float* state, con
   return launch_status();
 }
 
+template <int D, int E>
+int launch_decode_layer(const la::DecodeLayerArgs& a, int64_t nbh, cudaStream_t stream) {
+  la::decode_layer_kernel<D, E><<<static_cast<unsigned>(nbh), 256, 0, stream>>>(a);
+  return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -569,7 +577,7 @@ int lightning_attn_fwd_strided(const void* q, const void* k, const void* v, cons
                                const long long* k_strides, const long long* v_strides,
                                const long long* out_strides, int chunk, void* stream) {
   if (!q_strides || !k_strides || !v_strides || !out_strides) return LA_ERR_NULL;
-  Strides st;
+  Strides st = {};  // (the gate's entry is not used)
   const long long* src[4] = {q_strides, k_strides, v_strides, out_strides};
   for (int i = 0; i < 4; ++i)
     for (int j = 0; j < 3; ++j) st.s[i][j] = src[i][j];
@@ -606,6 +614,28 @@ int lightning_attn_fwd_fused(const void* q, const void* k, const void* v, const 
   const FusedArgs fa{gate, norm_weight, eps};
   return fwd_bf16_impl(q, k, v, slopes, nullptr, nullptr, out, B, H, N, D, E, 0, stream, nullptr,
                        false, 0, kWaitLimitNs, &fa);
+}
+
+int lightning_attn_fwd_fused_ex(const void* q, const void* k, const void* v, const void* gate,
+                                const float* slopes, const float* norm_weight, float eps,
+                                const float* init_state, float* final_state, void* out, int B,
+                                int H, int N, int D, int E, const long long* q_strides,
+                                const long long* k_strides, const long long* v_strides,
+                                const long long* gate_strides, const long long* out_strides,
+                                int chunk, void* stream) {
+  const FusedArgs fa{gate, norm_weight, eps};
+  const long long* src[5] = {q_strides, k_strides, v_strides, out_strides, gate_strides};
+  int given = 0;
+  for (const long long* x : src) given += x != nullptr;
+  if (given == 0)
+    return fwd_bf16_impl(q, k, v, slopes, init_state, final_state, out, B, H, N, D, E, chunk,
+                         stream, nullptr, false, 0, kWaitLimitNs, &fa);
+  if (given != 5) return LA_ERR_NULL;
+  Strides st;
+  for (int i = 0; i < 5; ++i)
+    for (int j = 0; j < 3; ++j) st.s[i][j] = src[i][j];
+  return fwd_bf16_impl(q, k, v, slopes, init_state, final_state, out, B, H, N, D, E, chunk,
+                       stream, &st, false, 0, kWaitLimitNs, &fa);
 }
 
 int lightning_attn_fault_test_scan_stall(const void* q, const void* k, const void* v,
@@ -652,6 +682,50 @@ int lightning_attn_decode(const void* q, const void* k, const void* v, float* st
   if (D == 128 && E == 64) return launch_decode<128, 64>(q, k, v, state, slopes, out, B, H, s);
   if (D == 128 && E == 128) return launch_decode<128, 128>(q, k, v, state, slopes, out, B, H, s);
   return LA_ERR_UNSUPPORTED;
+}
+
+int lightning_attn_decode_fused(const void* q, const void* k, const void* v, const void* gate,
+                                float* state, const float* slopes, const float* norm_weight,
+                                float eps, void* out, int B, int H, int D, int E,
+                                const long long* q_strides, const long long* k_strides,
+                                const long long* v_strides, const long long* gate_strides,
+                                const long long* out_strides, void* stream) {
+  if (!q || !k || !v || !gate || !state || !slopes || !norm_weight || !out) return LA_ERR_NULL;
+  if (!dims_ok(B, H, 1, D, E)) return LA_ERR_SHAPE;
+  if (!(eps >= 0.f) || eps > 3.0e38f) return LA_ERR_SHAPE;
+  if ((D != 64 && D != 128) || (E != 64 && E != 128)) return LA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) || !aligned16(state) ||
+      !aligned16(out) || !aligned4(slopes) || !aligned4(norm_weight))
+    return LA_ERR_ALIGN;
+  const long long* src[5] = {q_strides, k_strides, v_strides, gate_strides, out_strides};
+  int given = 0;
+  for (const long long* x : src) given += x != nullptr;
+  if (given != 0 && given != 5) return LA_ERR_NULL;
+  la::DecodeLayerArgs a{};
+  long long* dst[5] = {a.qs, a.ks, a.vs, a.gs, a.os};
+  const long long width[5] = {D, D, E, E, E};
+  for (int i = 0; i < 5; ++i) {
+    dst[i][0] = given ? src[i][0] : static_cast<long long>(H) * width[i];
+    dst[i][1] = given ? src[i][1] : width[i];
+    for (int j = 0; j < 2; ++j)  // 16-byte rows, as every other entry point's tensors
+      if (dst[i][j] < 0 || dst[i][j] % 8 != 0 || dst[i][j] >= (1ll << 40)) return LA_ERR_ALIGN;
+  }
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.gate = static_cast<const __nv_bfloat16*>(gate);
+  a.state = state;
+  a.slopes = slopes;
+  a.norm_w = norm_weight;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.eps = eps;
+  a.H = H;
+  const int64_t nbh = static_cast<int64_t>(B) * H;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 64 && E == 64) return launch_decode_layer<64, 64>(a, nbh, st);
+  if (D == 64 && E == 128) return launch_decode_layer<64, 128>(a, nbh, st);
+  if (D == 128 && E == 64) return launch_decode_layer<128, 64>(a, nbh, st);
+  return launch_decode_layer<128, 128>(a, nbh, st);
 }
 
 const char* lightning_attn_last_cuda_error(void) { return t_last_cuda_error; }

@@ -44,6 +44,10 @@ SIGNATURES = {
     "lightning_attn_fwd_strided": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P,
                                    _I, _P],
     "lightning_attn_set_cta_limit": [_I, _P],
+    "lightning_attn_fwd_fused_ex": [_P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P, _I, _I,
+                                    _I, _I, _I, _P, _P, _P, _P, _P, _I, _P],
+    "lightning_attn_decode_fused": [_P, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _I, _I, _I,
+                                    _I, _P, _P, _P, _P, _P, _P],
 }
 
 
@@ -248,6 +252,67 @@ def fwd_fused(q, k, v, gate, slopes, norm_weight, eps: float = 1e-6, out=None, *
                                         slopes.data_ptr(), norm_weight.data_ptr(), float(eps),
                                         out.data_ptr(), B, H, N, D, E, _stream_handle(stream))
     _check("lightning_attn_fwd_fused", rc)
+    return out
+
+
+@_on_tensor_device
+def fwd_fused_ex(q, k, v, gate, slopes, norm_weight, eps: float = 1e-6, out=None, *,
+                 init_state=None, final_state=None, chunk: int = 0, stream=None) -> torch.Tensor:
+    """The fused layer on [B,H,N,*] views with any (b, h, t) strides and a
+    contiguous last dimension (e.g. ``x.permute(0, 2, 1, 3)`` of token-major
+    [B,N,H,*] buffers, or slices of a fused [B,N,3,H,D] projection), with the
+    recurrent state (over the activated k, v) optionally handed in and out:
+    fp32 init_state / final_state [B,H,D,E].  out defaults to a head-major
+    contiguous bf16 tensor."""
+    B, H, N, D = q.shape
+    E = v.shape[-1]
+    _need_view(q, "q", torch.bfloat16, (B, H, N, D))
+    _need_view(k, "k", torch.bfloat16, (B, H, N, D))
+    _need_view(v, "v", torch.bfloat16, (B, H, N, E))
+    _need_view(gate, "gate", torch.bfloat16, (B, H, N, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    _need(norm_weight, "norm_weight", torch.float32, (H, E))
+    if out is None:
+        out = torch.empty((B, H, N, E), dtype=torch.bfloat16, device=q.device)
+    _need_view(out, "out", torch.bfloat16, (B, H, N, E))
+    for name, st in (("init_state", init_state), ("final_state", final_state)):
+        if st is not None:
+            _need(st, name, torch.float32, (B, H, D, E))
+    arr = [(ctypes.c_longlong * 3)(*t.stride()[:3]) for t in (q, k, v, gate, out)]
+    rc = lib().lightning_attn_fwd_fused_ex(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), gate.data_ptr(), slopes.data_ptr(),
+        norm_weight.data_ptr(), float(eps),
+        None if init_state is None else init_state.data_ptr(),
+        None if final_state is None else final_state.data_ptr(), out.data_ptr(), B, H, N, D, E,
+        *[ctypes.cast(a, ctypes.c_void_p) for a in arr], int(chunk), _stream_handle(stream))
+    _check("lightning_attn_fwd_fused_ex", rc)
+    return out
+
+
+@_on_tensor_device
+def decode_fused(q, k, v, gate, state, slopes, norm_weight, eps: float = 1e-6, out=None, *,
+                 stream=None) -> torch.Tensor:
+    """One decode step of the fused layer: raw bf16 q, k [B,H,D], v, gate [B,H,E]
+    views (any (b, h) strides, contiguous last dimension); fp32 state
+    [B,H,D,E] (contiguous) advanced in place; bf16 out [B,H,E]."""
+    B, H, D = q.shape
+    E = v.shape[-1]
+    _need_view(q, "q", torch.bfloat16, (B, H, D))
+    _need_view(k, "k", torch.bfloat16, (B, H, D))
+    _need_view(v, "v", torch.bfloat16, (B, H, E))
+    _need_view(gate, "gate", torch.bfloat16, (B, H, E))
+    _need(state, "state", torch.float32, (B, H, D, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    _need(norm_weight, "norm_weight", torch.float32, (H, E))
+    if out is None:
+        out = torch.empty((B, H, E), dtype=torch.bfloat16, device=q.device)
+    _need_view(out, "out", torch.bfloat16, (B, H, E))
+    arr = [(ctypes.c_longlong * 2)(*t.stride()[:2]) for t in (q, k, v, gate, out)]
+    rc = lib().lightning_attn_decode_fused(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), gate.data_ptr(), state.data_ptr(),
+        slopes.data_ptr(), norm_weight.data_ptr(), float(eps), out.data_ptr(), B, H, D, E,
+        *[ctypes.cast(a, ctypes.c_void_p) for a in arr], _stream_handle(stream))
+    _check("lightning_attn_decode_fused", rc)
     return out
 
 

@@ -100,8 +100,8 @@ def test_binding_runs_each_entry_on_its_tensors_device():
     # every entry point is wrapped so it launches on the device of its tensors
     # and refuses tensors spread over devices (checked with real devices on GPU
     # boxes; here the wrapper's pass-through for non-CUDA tensors)
-    for name in ("fwd", "fwd_strided", "fwd_anticausal", "fwd_fused", "bwd", "fwd_noalloc",
-                 "fwd_f32", "decode", "fault_test_scan_stall"):
+    for name in ("fwd", "fwd_strided", "fwd_anticausal", "fwd_fused", "fwd_fused_ex", "bwd",
+                 "fwd_noalloc", "fwd_f32", "decode", "decode_fused", "fault_test_scan_stall"):
         fn = getattr(ops, name)
         assert getattr(fn, "__wrapped__", None) is not None, name
     import torch
@@ -177,3 +177,24 @@ def test_cta_limit_setter(lib):
         assert ops.set_cta_limit(0) == 0  # a rejected call leaves the cap alone
     finally:
         ops.set_cta_limit(prev)
+
+
+def test_fused_ex_and_decode_fused_validation(lib):
+    C3, C2 = ctypes.c_longlong * 3, ctypes.c_longlong * 2
+    f = lib.lightning_attn_fwd_fused_ex
+    st = C3(64 * 8 * 128, 128, 8 * 128)
+    args = lambda eps, strides: (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, eps, None, None, FAKE, 1, 8,
+                                 64, 128, 128, *strides, 0, None)
+    assert f(*args(1e-6, (st, st, None, st, st))) == LA_ERR_NULL  # strides: all or none
+    assert f(*args(-1.0, (None,) * 5)) == LA_ERR_SHAPE
+    bad = C3(64 * 8 * 128, 128, 8 * 128 + 4)  # 8-byte token stride
+    assert f(*args(1e-6, (st, st, st, bad, st))) == LA_ERR_ALIGN
+    g = lib.lightning_attn_decode_fused
+    s2 = C2(8 * 128, 128)
+    dargs = lambda eps, strides, D=128: (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, eps, FAKE, 2, 8,
+                                         D, 128, *strides, None)
+    assert g(*dargs(1e-6, (s2, None, s2, s2, s2))) == LA_ERR_NULL
+    assert g(*dargs(float("nan"), (None,) * 5)) == LA_ERR_SHAPE
+    assert g(*dargs(1e-6, (None,) * 5, D=96)) == LA_ERR_UNSUPPORTED
+    assert g(*dargs(1e-6, (s2, s2, s2, C2(8 * 128, 132), s2))) == LA_ERR_ALIGN
+    assert g(None, *dargs(1e-6, (None,) * 5)[1:]) == LA_ERR_NULL
