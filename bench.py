@@ -426,7 +426,11 @@ def bench_prefill(args, dist, w, dev):
     return res
 
 
-def bench_decode(args, dist, dev):
+def bench_decode(args, dist, dev, fused: bool = False):
+    """1024 chained decode steps of the decode workload (256 sequences x 64
+    heads, fp32 128x128 states), inputs resident on the device.  fused: the
+    layer's decode step (lightning_attn_decode_fused: raw q, k, v and gate in,
+    SiLU, state step, RMSNorm, weight and sigmoid gate, bf16 out)."""
     import torch
     from long_context_fwd_b200 import inputs as I
     from long_context_fwd_b200 import ops
@@ -437,26 +441,41 @@ def bench_decode(args, dist, dev):
     g.manual_seed(4321)
     state = torch.randn((w.B, w.H, w.D, w.E), generator=g, device=dev) * 0.02
     sl = torch.from_numpy(I.slopes_for(w)).to(dev)
-    qs = torch.nn.functional.silu(torch.randn((steps, w.B, w.H, w.D), generator=g, device=dev)).to(torch.bfloat16)
-    ks = torch.nn.functional.silu(torch.randn((steps, w.B, w.H, w.D), generator=g, device=dev)).to(torch.bfloat16)
+    act = (lambda x: x) if fused else torch.nn.functional.silu
+    qs = act(torch.randn((steps, w.B, w.H, w.D), generator=g, device=dev)).to(torch.bfloat16)
+    ks = act(torch.randn((steps, w.B, w.H, w.D), generator=g, device=dev)).to(torch.bfloat16)
     vs = torch.randn((steps, w.B, w.H, w.E), generator=g, device=dev).to(torch.bfloat16)
-    out = torch.empty((w.B, w.H, w.E), dtype=torch.float32, device=dev)
+    if fused:
+        gs = torch.randn((steps, w.B, w.H, w.E), generator=g, device=dev).to(torch.bfloat16)
+        nw = torch.ones((w.H, w.E), dtype=torch.float32, device=dev)
+        out = torch.empty((w.B, w.H, w.E), dtype=torch.bfloat16, device=dev)
+        step = lambda i: ops.decode_fused(qs[i], ks[i], vs[i], gs[i], state, sl, nw, 1e-6, out)
+    else:
+        out = torch.empty((w.B, w.H, w.E), dtype=torch.float32, device=dev)
+        step = lambda i: ops.decode(qs[i], ks[i], vs[i], state, sl, out)
     stream = torch.cuda.current_stream()
     for i in range(max(3, args.warmup)):
-        ops.decode(qs[i % steps], ks[i % steps], vs[i % steps], state, sl, out)
+        step(i % steps)
     torch.cuda.synchronize()
     dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_host0 = time.time()
     e0.record(stream)
     for i in range(steps):
-        ops.decode(qs[i], ks[i], vs[i], state, sl, out)
+        step(i)
     e1.record(stream)
     torch.cuda.synchronize()
     t_host1 = time.time()
     dist.barrier()
     ms = dist.max(e0.elapsed_time(e1)) / steps
-    bytes_step = w.B * w.H * (2 * w.D * w.E * 4 + 2 * w.D * 2 + 2 * w.E + 4 * w.E + 4)
+    if fused:
+        # state read + write (fp32), q, k, v and gate in (bf16), out (bf16), the
+        # slope; the norm weight [H][E] once per step
+        bytes_step = (w.B * w.H * (2 * w.D * w.E * 4 + 2 * w.D * 2 + 2 * w.E + 2 * w.E + 4) +
+                      w.H * w.E * 4)
+        del gs
+    else:
+        bytes_step = w.B * w.H * (2 * w.D * w.E * 4 + 2 * w.D * 2 + 2 * w.E + 4 * w.E + 4)
     finite = bool(torch.isfinite(state).all().item())
     del qs, ks, vs, state
     torch.cuda.empty_cache()
@@ -619,6 +638,7 @@ def main_ours(args):
                                                     max(1e-3, prefill_bytes(wx) / hbm / 1e6))))
         legs[name] = (wx, bench_prefill_leg(dist, wx, dev, steps, args.warmup))
     dec = None if args.no_decode else bench_decode(args, dist, dev)
+    decf = None if args.no_decode else bench_decode(args, dist, dev, fused=True)
     bwd = None if args.backward_steps <= 0 else bench_backward(args, dist, w, dev)
     fus = None if args.fused_steps <= 0 else bench_fused(args, dist, w, dev)
     sampler.stop()
@@ -699,6 +719,17 @@ def main_ours(args):
                           "clocks": sampler.summary([dec["window"]]),
                           "roofline": roofline(dec["bytes"], dec["flops"], dec["ms"], hbm, bf16,
                                                None, peak_src)}
+    if decf:
+        line["decode_layer"] = {"workload": decf["workload"],
+                                "what": "lightning_attn_decode_fused: SiLU on raw q, k, v, the "
+                                        "state step, RMSNorm, weight and sigmoid gate, bf16 out",
+                                "value": dist.world * decf["tokens"] / (decf["ms"] / 1e3),
+                                "unit": "tokens/s", "ms_per_step": decf["ms"],
+                                "steps": decf["steps"], "gpu_launches": decf["steps"],
+                                "state_finite": decf["finite"],
+                                "clocks": sampler.summary([decf["window"]]),
+                                "roofline": roofline(decf["bytes"], decf["flops"], decf["ms"], hbm,
+                                                     bf16, None, peak_src)}
     if bwd:
         # minimal traffic of the operation: q, k, v, dout read once (bf16), dq,
         # dk, dv written once (fp32); flops: three launches of the blocked form
