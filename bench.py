@@ -119,6 +119,8 @@ def parse():
                     help="prefill q/k/v/out layout: [B][H][N][D] or [B][N][H][D]")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the end-to-end leg")
+    ap.add_argument("--e2e-upload-streams", type=int, default=2,
+                    help="streams the end-to-end leg's uploads alternate between")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="0 skips the CPU baseline")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--backward-steps", type=int, default=20,
@@ -357,15 +359,17 @@ def bench_prefill(args, dist, w, dev):
     dq, dk, dv = (torch.empty(x.shape, dtype=x.dtype, device=dev) for x in (hq, hk, hv))
 
     # The step runs as G groups of consecutive (b, h) sequences (whole batch rows,
-    # or equal runs of heads of one row): one stream copies every group's inputs
-    # up back to back, one runs each group's prefill once its inputs are in, one
-    # copies each group's result down once it is computed, so uploads run
-    # continuously and overlap the downloads (PCIe is full duplex).
+    # or equal runs of heads of one row): upload streams (groups taken in turn)
+    # copy every group's inputs up back to back, one stream runs each group's
+    # prefill once its inputs are in, one copies each group's result down once
+    # it is computed, so uploads run continuously and overlap the downloads
+    # (PCIe is full duplex).
     nseq = w.B * w.H
     G = next((g for g in (16, 8, 4, 2) if nseq % g == 0 and
               (w.H % (nseq // g) == 0 or (nseq // g) % w.H == 0)), 1)
     per = nseq // G
-    up, comp, down = (torch.cuda.Stream(device=dev) for _ in range(3))
+    ups = [torch.cuda.Stream(device=dev) for _ in range(max(1, args.e2e_upload_streams))]
+    comp, down = (torch.cuda.Stream(device=dev) for _ in range(2))
 
     def group_views(i):
         lo = i * per
@@ -385,11 +389,12 @@ def bench_prefill(args, dist, w, dev):
             return
         start = torch.cuda.Event()
         start.record(stream)
-        for st in (up, comp, down):
+        for st in (*ups, comp, down):
             st.wait_event(start)
         for i in range(G):
             shp, hs = group_views(i)
             gq, gk, gv, go = shp(dq), shp(dk), shp(dv), shp(out)
+            up = ups[i % len(ups)]
             with torch.cuda.stream(up):
                 gq.copy_(shp(hq), non_blocking=True)
                 gk.copy_(shp(hk), non_blocking=True)
@@ -679,8 +684,9 @@ def main_ours(args):
             "value": job_throughput(dist.world, tokens_step, pre["e2e_ms"]), "unit": "tokens/s",
             "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"],
             "ms_per_step": pre["e2e_ms"],
-            "pipelining": f"{pre['e2e_groups']} groups of sequences: uploads, prefills and "
-                          "downloads on three streams, ordered per group by events"},
+            "pipelining": f"{pre['e2e_groups']} groups of sequences: uploads on "
+                          f"{args.e2e_upload_streams} stream(s), prefills and downloads on one "
+                          "each, ordered per group by events"},
         "clocks": sampler.summary([pre["window"]]),
     }
     if "sustained" in pre:
