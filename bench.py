@@ -119,8 +119,9 @@ def parse():
                     help="prefill q/k/v/out layout: [B][H][N][D] or [B][N][H][D]")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the end-to-end leg")
-    ap.add_argument("--e2e-upload-streams", type=int, default=2,
-                    help="streams the end-to-end leg's uploads alternate between")
+    ap.add_argument("--e2e-upload-streams", type=int, default=1,
+                    help="streams the end-to-end leg's uploads alternate between (two measured "
+                         "slower: 146 vs 134-136 ms per step)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="0 skips the CPU baseline")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--backward-steps", type=int, default=20,

@@ -129,8 +129,9 @@ int lightning_attn_fwd_ex(const void* q, const void* k, const void* v,
  * state slot -- 2 B H slots for the chunk scan, at most 2 per SM for the
  * automatic splits.  A call
  * that would need more than LA_NOALLOC_SCRATCH_BYTES returns LA_ERR_WORKSPACE
- * before launching anything.  With chunk = 0 the split is only used when B*H
- * is below the SM count, which stays within the limit on a 148-SM B200.
+ * before launching anything.  With chunk = 0 the automatic splits need at most
+ * two states per CTA (19.4 MB on a 148-SM B200), within the limit; on a GPU
+ * with so many SMs that they would not fit, the call runs whole sequences.
  * The first call on each device loads the library's device code and looks up
  * the array's device address (cudaGetSymbolAddress); make that first call
  * before any stream capture.  The address is looked up again on every call

@@ -145,3 +145,49 @@ def test_decode_layer_chain_from_random_states(D, E):
         assert rel(y.float().cpu().numpy(), ref[:, :, 0]) <= TOL_BF16
     _done()
     assert rel(state.cpu().numpy(), sref) <= 1e-4
+
+
+@pytest.mark.parametrize("D,E", [(64, 64), (64, 128), (128, 64)])
+def test_token_major_layer_narrow_heads_with_state(D, E):
+    # 64-wide heads through the 4-D tensor maps (zero-filled second halves),
+    # token-major in and out, with an initial state and the final state
+    B, H, N = 2, 3, 1000
+    q, k, v, g, w, sl = _case(B, H, N, D, E, seed=D + 2 * E)
+    s0 = (0.05 * np.random.default_rng(D * E).standard_normal((B, H, D, E))).astype(np.float32)
+    views = [_token_major(x)[1] for x in (q, k, v, g)]
+    out_buf = torch.empty((B, N, H, E), dtype=torch.bfloat16, device=DEV)
+    fin = torch.empty((B, H, D, E), dtype=torch.float32, device=DEV)
+    ops.fwd_fused_ex(*views, f32_to_dev(sl, DEV), f32_to_dev(w, DEV), 1e-6,
+                     out_buf.permute(0, 2, 1, 3), init_state=f32_to_dev(s0, DEV), final_state=fin)
+    _done()
+    ref, sref = oracle.fused_layer(q, k, v, g, sl, w, 1e-6, s0=s0.astype(np.float64),
+                                   return_state=True)
+    got = out_buf.permute(0, 2, 1, 3).float().cpu().numpy()
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+    assert rel(fin.cpu().numpy(), sref) <= TOL_BF16
+
+
+def test_decode_layer_strided_output_rows():
+    # the step's output written into every other row of a wider buffer
+    # (strides {2 H E, E}), inputs token-major slices of one [B, H, 4, 128] row
+    B, H, D, E = 4, 6, 128, 128
+    w_ = I.Workload("declayer_s", B, H, 1, D, E, "bf16", steps=1, kind="decode", index=97)
+    s0 = I.decode_state(w_)
+    rng = np.random.default_rng(11)
+    raw = I.f32_to_bf16_bits(rng.standard_normal((B, H, 4, 128)).astype(np.float32))
+    buf = bf16_to_dev(raw, DEV)
+    w = (1.0 + 0.25 * rng.standard_normal((H, E))).astype(np.float32)
+    sl = I.alibi_slopes(H)
+    state = f32_to_dev(s0, DEV)
+    wide = torch.zeros((B, 2 * H, E), dtype=torch.bfloat16, device=DEV)
+    outv = wide[:, ::2]
+    ops.decode_fused(buf[:, :, 0], buf[:, :, 1], buf[:, :, 2], buf[:, :, 3], state,
+                     f32_to_dev(sl, DEV), f32_to_dev(w, DEV), 1e-6, outv)
+    _done()
+    q, k, v, g = (np.ascontiguousarray(raw[:, :, i])[:, :, None] for i in range(4))
+    ref, sref = oracle.fused_layer(q, k, v, g, sl, w, 1e-6, s0=s0.astype(np.float64),
+                                   return_state=True)
+    assert rel(outv.float().cpu().numpy(), ref[:, :, 0]) <= TOL_BF16
+    assert torch.all(wide[:, 1::2] == 0)
+    assert rel(state.cpu().numpy(), sref) <= 1e-4

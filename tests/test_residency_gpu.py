@@ -80,3 +80,31 @@ def test_two_streams_without_ordering(B, H, N):
     for (q, k, v, sl), o in zip(cases, outs):
         ref = oracle.recurrent(q, k, v, sl)
         assert rel(o.cpu().numpy(), ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("entry", ["fused", "anticausal", "noalloc"])
+def test_other_entries_on_a_capped_grid(entry, cta_limit):
+    # the fused layer, the reverse-time operator and the allocation-free entry
+    # plan their splits for the capped grid too (split scan at 40 CTAs)
+    B, H, N = 1, 24, 3000
+    assert ops.fwd_plan(B, H, N, 0, 40)[0]["mode"] == 2
+    q, k, v, sl = _case(7, B, H, N)
+    cta_limit(40)
+    tq, tk, tv = (bf16_to_dev(x, DEV) for x in (q, k, v))
+    ts = f32_to_dev(sl, DEV)
+    if entry == "fused":
+        g = I.f32_to_bf16_bits(np.random.default_rng(3).standard_normal(q.shape).astype(np.float32))
+        w = np.ones((H, 128), np.float32)
+        got = ops.fwd_fused(tq, tk, tv, bf16_to_dev(g, DEV), ts, f32_to_dev(w, DEV), 1e-6)
+        ref = oracle.fused_layer(q, k, v, g, sl, w, 1e-6)
+    elif entry == "anticausal":
+        got = ops.fwd_anticausal(tq, tk, tv, ts)
+        ref = oracle.recurrent_anticausal(q, k, v, sl)
+    else:
+        got = ops.fwd_noalloc(tq, tk, tv, ts)
+        ref = oracle.recurrent(q, k, v, sl)
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0
+    got = got.float().cpu().numpy()
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
