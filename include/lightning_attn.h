@@ -277,6 +277,8 @@ int lightning_attn_fwd_fused(const void* q, const void* k, const void* v, const 
  *                H*W}; slices of one fused [B][N][3][H][D] projection output
  *                {3*N*H*D, D, 3*H*D}.  Every stride times 2 bytes a multiple of
  *                16 below 2^40, every pointer 16-byte aligned (LA_ERR_ALIGN).
+ *                The elements of out must not overlap each other or the inputs
+ *                (not checked).
  *   chunk      : as lightning_attn_fwd_ex.
  * Everything else -- the computation, eps, norm_weight [H][E], bf16 out,
  * D, E in {64, 128}, the errors -- as lightning_attn_fwd_fused.
