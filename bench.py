@@ -134,6 +134,8 @@ def parse():
     ap.add_argument("--extra-workloads",
                     default="prefill_b1h64n8192d128,prefill_b1h64n1048576d128",
                     help="comma-separated prefill workloads timed as legs of the same line")
+    ap.add_argument("--state-workloads", default="prefill_b1h64n1048576d128",
+                    help="comma-separated workloads whose state pass alone is timed as a leg")
     ap.add_argument("--extra-seconds", type=float, default=0.5,
                     help="about this much roofline time per extra leg")
     ap.add_argument("--extra-max-steps", type=int, default=300)
@@ -309,6 +311,28 @@ def bench_prefill_leg(dist, w, dev, steps: int, warmup: int) -> dict:
     assert ops.device_status(reset=True) == 0, "device-side wait timed out during warm-up"
     res = timed_launches(dist, stream, steps, lambda: ops.fwd(q, k, v, sl, out))
     del q, k, v, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_state_leg(dist, w, dev, steps: int, warmup: int) -> dict:
+    """The state pass alone (lightning_attn_state: K and V in, the state after
+    the sequence out) on a prefill workload's shapes, inputs resident."""
+    import torch
+    from long_context_fwd_b200 import inputs as I
+    from long_context_fwd_b200 import ops
+
+    _, k, v = I.device_prefill_inputs(w, dev)  # (q is drawn and dropped: same k, v as the prefill)
+    torch.cuda.empty_cache()
+    sl = torch.from_numpy(I.slopes_for(w)).to(dev)
+    st = torch.empty((w.B, w.H, w.D, w.E), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, warmup)):
+        ops.state(k, v, sl, st)
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0, "device-side wait timed out during warm-up"
+    res = timed_launches(dist, stream, steps, lambda: ops.state(k, v, sl, st))
+    del k, v, st
     torch.cuda.empty_cache()
     return res
 
@@ -643,6 +667,13 @@ def main_ours(args):
         steps = max(3, min(args.extra_max_steps, int(args.extra_seconds * 1e3 /
                                                     max(1e-3, prefill_bytes(wx) / hbm / 1e6))))
         legs[name] = (wx, bench_prefill_leg(dist, wx, dev, steps, args.warmup))
+    states = {}
+    for name in [x for x in args.state_workloads.split(",") if x]:
+        wx = I.WORKLOADS[name]
+        sbytes = wx.B * wx.H * wx.N * 2 * (wx.D + wx.E)
+        steps = max(3, min(args.extra_max_steps, int(args.extra_seconds * 1e3 /
+                                                    max(1e-3, sbytes / hbm / 1e6))))
+        states[name] = (wx, bench_state_leg(dist, wx, dev, steps, args.warmup))
     dec = None if args.no_decode else bench_decode(args, dist, dev)
     decf = None if args.no_decode else bench_decode(args, dist, dev, fused=True)
     bwd = None if args.backward_steps <= 0 else bench_backward(args, dist, w, dev)
@@ -716,6 +747,19 @@ def main_ours(args):
             "clocks": sampler.summary([r["window"]]),
             "roofline": roofline(prefill_bytes(wx), prefill_flops(wx), r["launch_ms"], hbm, bf16,
                                  traffic_for(wx), peak_src)}
+    for name, (wx, r) in states.items():
+        # k and v read once (bf16), the state written once (fp32); flops: the
+        # state product (K~^T V) per token-head
+        sbytes = wx.B * wx.H * (wx.N * 2 * (wx.D + wx.E) + 4 * wx.D * wx.E)
+        line["state_" + {8192: "8k", 1 << 20: "1m"}.get(wx.N, wx.name)] = {
+            "workload": wx.name, "what": "lightning_attn_state: the state after the sequence, "
+                                         "no outputs (prompt prefix / sequence-split step)",
+            "value": job_throughput(dist.world, wx.B * wx.N, r["total_ms"] / r["steps"]),
+            "unit": "tokens/s", "steps": r["steps"], "ms_per_step": r["total_ms"] / r["steps"],
+            "gpu_launches": r["steps"], "device_status": r["status"],
+            "clocks": sampler.summary([r["window"]]),
+            "roofline": roofline(sbytes, wx.B * wx.H * wx.N * 2 * wx.D * wx.E, r["launch_ms"],
+                                 hbm, bf16, None, peak_src)}
     if dec:
         # per head-step: the state read and written (fp32), q, k, v in (bf16),
         # out (fp32) and the slope; flops: decay, k^T v and q S, 5 D E

@@ -317,6 +317,51 @@ int lightning_attn_decode_fused(const void* q, const void* k, const void* v, con
                                 const long long* out_strides, void* stream);
 
 /*
+ * The state pass alone: the recurrent state after N tokens,
+ *   final_state = exp(-lambda N) S_0 + sum_t exp(-lambda (N-1-t)) k_t^T v_t,
+ * without the outputs ("MiniMax-M1" model entry: the linear layers' fixed-size
+ * recurrent state, 128x128 per head).  Reads only k and v (512 B per
+ * token-head at D = E = 128 instead of the prefill's 1280): for a prompt prefix
+ * whose outputs are not needed (the state is what a later prefill or decode
+ * continues from), and for the per-chunk states of a sequence split across
+ * GPUs (lightning_attn_state_combine).
+ *   k : bf16 [B][H][N][D]     v : bf16 [B][H][N][E]    slopes: fp32 [H]
+ *   init_state : nullable fp32 [B][H][D][E] (S_0; zero if NULL)
+ *   final_state: fp32 [B][H][D][E], fully overwritten (required)
+ *   chunk      : as lightning_attn_fwd_ex; 0 picks whole sequences when B*H
+ *                fills the grid, else chunks of 1024-8192 tokens chained by
+ *                a ticketed scan (scratch from cudaMallocAsync on `stream`)
+ * Runs the prefill kernel's local-state pass (tcgen05 K~^T V products into a
+ * TMEM state).  D, E in {64, 128}; errors as lightning_attn_fwd.
+ */
+int lightning_attn_state(const void* k, const void* v, const float* slopes,
+                         const float* init_state, float* final_state, int B, int H, int N, int D,
+                         int E, int chunk, void* stream);
+
+/*
+ * Combines the states of R consecutive chunks of B*H sequences into the state
+ * after all of them: with L_j the state of chunk j (n_j tokens) from a zero
+ * initial state (lightning_attn_state, init_state NULL),
+ *   out = gamma^(n_0 + ... + n_{R-1}) S_0 + sum_j gamma^(n_{j+1} + ... + n_{R-1}) L_j
+ * (gamma = exp(-lambda_h); the recurrence is linear in its initial state).
+ * This is the one exchange step of a sequence split across GPUs (the
+ * abstract's 4M-token inference context): each rank computes L_r of its own
+ * chunk, the L_r are all-gathered, and rank r combines L_0 .. L_{r-1} into the
+ * entering state of its prefill (lightning_attn_fwd_ex init_state).
+ *   states      : fp32 [R][B][H][D][E] (nullable if R = 0), the layout of an
+ *                 all-gather of [B][H][D][E] tensors
+ *   R           : 0 .. 256 (LA_ERR_SHAPE beyond)
+ *   chunk_tokens: HOST array of R token counts (>= 0)
+ *   init_state  : nullable fp32 [B][H][D][E] (S_0; zero if NULL)
+ *   out         : fp32 [B][H][D][E]; must not overlap the inputs
+ * One CUDA-core kernel, HBM-bound (R + 1 states read, one written).
+ * D, E in {64, 128}; 16-byte aligned state pointers (LA_ERR_ALIGN).
+ */
+int lightning_attn_state_combine(const float* states, int R, const int* chunk_tokens,
+                                 const float* slopes, const float* init_state, float* out, int B,
+                                 int H, int D, int E, void* stream);
+
+/*
  * Fault-injection hook for testing the bounded device-side waits (an interface
  * for tests; the pages have no counterpart).  Runs the chunked bf16 prefill
  * (D = E = 128, chunk a multiple of 128 with N > chunk) but hands out work

@@ -709,8 +709,16 @@ __device__ void group_x(const Ctx& c, const Params& p) {
           qv[4 * ch + 2] = scale_bf16x2(x.z, fq);
           qv[4 * ch + 3] = scale_bf16x2(x.w, fq);
         }
-        warp_arrive(&c.bar[B_QE + qs]);
         tmem_st32(t_s + 32u, qv);
+        // The Q tile is dead now.  Its release comes after the TMEM store
+        // (which consumes every load above, so they have completed) and a
+        // proxy fence (these generic-proxy reads are ordered before the TMA
+        // write of a later tile into the slot, an async-proxy access): when the
+        // release came straight after the loads, the producer's next Q tile
+        // could land while a warp's reads were still in flight, and the inter
+        // term of that warp's rows then used rows of the wrong tile.
+        fence_proxy_async_smem();
+        warp_arrive(&c.bar[B_QE + qs]);
       }
       // gamma^(len-1-r) K (0 past len) in place
       // gamma^(len-1-j) for the local index j of row r (0 past len)
@@ -856,8 +864,9 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
       if (!chain) scan_src = p.prefix + static_cast<int64_t>(it.enter_slot) * (HD * HD);
     }
     // the caller's initial state enters at block 0 of a sequence (or through
-    // the chain); never into a local state
-    if (p.init_state && it.p2 && (!it.enter || chain) && row_in)
+    // the chain); never into a local state -- except in the state pass, where
+    // the first chunk's inclusive state starts from it
+    if (p.init_state && (it.p2 || p.state_only) && (!it.enter || chain) && row_in)
       init_src = p.init_state + static_cast<int64_t>(it.seq) * state_elems + row_off;
     if (leader) LA_TRACE_EVENT(16, w_it);
     if (it.phase1 && !cwait(c, p, B_AGG_FULL, agg_n++ & 1u)) break;
@@ -901,7 +910,14 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             agg[i] = __float_as_uint(fmaf(gL, __uint_as_float(prev[i]), __uint_as_float(agg[i])));
-          st_scan32(pub, r, q >> 1, q & 1u, agg);
+          if (p.state_only && it.last) {  // the state after the sequence, to the caller
+            if (row_in && 32 * static_cast<int>(q) < p.E)
+              st_global32(p.final_state + static_cast<int64_t>(it.seq) * state_elems + row_off +
+                              32 * q,
+                          agg);
+          } else {
+            st_scan32(pub, r, q >> 1, q & 1u, agg);
+          }
         }
         if (it.p2) {
           store_half_bf16(kvb_row(q), r, q & 1u, prev, 1.f);
@@ -910,7 +926,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
       }
     }
     if (leader) LA_TRACE_EVENT(18, w_it);
-    if (it.phase1) {
+    if (it.phase1 && !(p.state_only && it.last)) {  // (the state pass's last chunk has no successor)
       // the group's stores are ordered before the leader's fence and release
       if (!gsync(c, p, B_YSYNC, ys_n)) break;
       if (leader) {

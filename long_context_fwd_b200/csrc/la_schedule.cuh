@@ -30,6 +30,8 @@ struct Params {
   int H, N, nseq, L, nchunks, total;
   int ticket_base;            // first ticket handed out (0 except in fault-injection runs)
   int mode;                   // work items: MODE_TICKETS, MODE_HANDOVER or MODE_SPLIT_SCAN
+  int state_only;             // the state pass alone (lightning_attn_state): every chunk a
+                              // local-state item, no outputs; the last writes final_state
   int nblk;                   // 128-token blocks per sequence
   int F, G2;                  // split scan: blocks of each sequence in the local-state pass;
                               // CTAs whose outputs cover that part
@@ -78,8 +80,8 @@ LA_HD Item decode_item(const Params& p, int w) {
   it.t0 = it.chunk * p.L;
   it.Lc = la_min(p.L, p.N - it.t0);
   it.nb = (it.Lc + BLK - 1) / BLK;
-  it.phase1 = it.chunk + 1 < p.nchunks;
-  it.p2 = true;
+  it.phase1 = p.state_only || it.chunk + 1 < p.nchunks;
+  it.p2 = !p.state_only;
   it.publish = false;
   it.enter = it.chunk > 0;
   it.last = it.chunk + 1 == p.nchunks;

@@ -23,6 +23,7 @@ __device__ int g_status;
 #include "la_decode.cuh"
 #include "la_fwd_f32.cuh"
 #include "la_fwd_sm100.cuh"
+#include "la_state.cuh"
 
 namespace {
 
@@ -193,6 +194,38 @@ Plan make_plan(int nseq, int N, int sms, int chunk) {
   pl.total = static_cast<long long>(nseq) * pl.nchunks;
   pl.grid = static_cast<int>(pl.total < sms ? pl.total : sms);
   if (pl.nchunks > 1) {
+    pl.ctrl = ctrl_bytes(static_cast<size_t>(nseq) * 2);
+    pl.bytes = pl.ctrl + static_cast<size_t>(nseq) * 2 * state_bytes;
+  }
+  return pl;
+}
+
+// The state pass (lightning_attn_state): every chunk a local-state item of the
+// ticketed chunk scan, the last one of each sequence writing the caller's
+// final state.  Whole sequences when there are enough of them to fill the
+// grid; otherwise chunks of 1024-8192 tokens, about four items per CTA.
+Plan make_state_plan(int nseq, int N, int sms, int chunk) {
+  Plan pl;
+  const int nblk = (N + 127) / 128;
+  pl.nblk = nblk;
+  pl.mode = la::fwd::MODE_TICKETS;
+  int L = chunk;
+  if (L == 0) {
+    L = nblk * 128;
+    if (nseq < sms && nblk > 8) {
+      const int want_chunks = (4 * sms + nseq - 1) / nseq;
+      L = ((N + want_chunks - 1) / want_chunks + 127) / 128 * 128;
+      if (L < 1024) L = 1024;
+      if (L > 8192) L = 8192;
+    }
+  }
+  if (L > nblk * 128) L = nblk * 128;
+  pl.L = L;
+  pl.nchunks = (N + L - 1) / L;
+  pl.total = static_cast<long long>(nseq) * pl.nchunks;
+  pl.grid = static_cast<int>(pl.total < sms ? pl.total : sms);
+  if (pl.nchunks > 1) {
+    const size_t state_bytes = 128 * 128 * sizeof(float);
     pl.ctrl = ctrl_bytes(static_cast<size_t>(nseq) * 2);
     pl.bytes = pl.ctrl + static_cast<size_t>(nseq) * 2 * state_bytes;
   }
@@ -549,6 +582,63 @@ int launch_decode(const void* q, const void* k, const void* v, float* state, con
   return launch_status();
 }
 
+int state_impl(const void* k, const void* v, const float* slopes, const float* init_state,
+               float* final_state, int B, int H, int N, int D, int E, int chunk,
+               void* stream_ptr) {
+  if (!k || !v || !slopes || !final_state) return LA_ERR_NULL;
+  if (!dims_ok(B, H, N, D, E)) return LA_ERR_SHAPE;
+  if ((D != 64 && D != 128) || (E != 64 && E != 128)) return LA_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(v) || !aligned4(slopes) || !aligned16(final_state) ||
+      (init_state && !aligned16(init_state)))
+    return LA_ERR_ALIGN;
+  if (chunk < 0 || (chunk % 128) != 0) return LA_ERR_SHAPE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  const int nseq = B * H;
+  la::fwd::Params p{};
+  CUtensorMap tk, tv;
+  const uint64_t ns = static_cast<uint64_t>(nseq);
+  if (!la::make_tmap_3d(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, N, ns, 64, 128) ||
+      !la::make_tmap_3d(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, E, N, ns, 64, 128))
+    return LA_ERR_CUDA;
+  p.D = D;
+  p.E = E;
+  const FwdKernel kern = pick_fwd_kernel(3, false, false);
+  int ctas = 0;
+  int rc = prepare_fwd_kernel(kern, &ctas);
+  if (rc != LA_OK) return rc;
+  const Plan pl = make_state_plan(nseq, N, ctas, chunk);
+  if (pl.total >= (1ll << 31)) return LA_ERR_SHAPE;
+  p.slopes = slopes;
+  p.init_state = init_state;
+  p.final_state = final_state;
+  p.state_only = 1;
+  p.status = status_word();
+  if (!p.status) return LA_ERR_CUDA;
+  p.H = H;
+  p.N = N;
+  apply_plan(pl, nseq, p);
+  p.wait_limit_ns = kWaitLimitNs;
+  p.tag = launch_tag();
+  void* scratch = nullptr;
+  if (pl.bytes) {
+    cudaError_t e = cudaMallocAsync(&scratch, pl.bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaMemsetAsync(scratch, 0, pl.ctrl, stream);  // the ticket and chunk flags
+    if (e != cudaSuccess) {
+      cudaFreeAsync(scratch, stream);
+      return cuda_fail(e);
+    }
+    set_scratch(pl, scratch, p);
+  }
+  // q and out take no part in the state pass: the K map stands in for both
+  rc = launch_fwd(kern, pl.grid, false, stream, tk, tk, tv, tk, p);
+  if (scratch) {
+    const cudaError_t e = cudaFreeAsync(scratch, stream);
+    if (e != cudaSuccess && rc == LA_OK) rc = cuda_fail(e);
+  }
+  return rc;
+}
+
 template <int D, int E>
 int launch_decode_layer(const la::DecodeLayerArgs& a, int64_t nbh, cudaStream_t stream) {
   la::decode_layer_kernel<D, E><<<static_cast<unsigned>(nbh), 256, 0, stream>>>(a);
@@ -726,6 +816,40 @@ int lightning_attn_decode_fused(const void* q, const void* k, const void* v, con
   if (D == 64 && E == 128) return launch_decode_layer<64, 128>(a, nbh, st);
   if (D == 128 && E == 64) return launch_decode_layer<128, 64>(a, nbh, st);
   return launch_decode_layer<128, 128>(a, nbh, st);
+}
+
+int lightning_attn_state(const void* k, const void* v, const float* slopes,
+                         const float* init_state, float* final_state, int B, int H, int N, int D,
+                         int E, int chunk, void* stream) {
+  return state_impl(k, v, slopes, init_state, final_state, B, H, N, D, E, chunk, stream);
+}
+
+int lightning_attn_state_combine(const float* states, int R, const int* chunk_tokens,
+                                 const float* slopes, const float* init_state, float* out, int B,
+                                 int H, int D, int E, void* stream) {
+  if (!slopes || !out || (R > 0 && (!states || !chunk_tokens))) return LA_ERR_NULL;
+  if (R < 0 || R > la::COMBINE_MAX_CHUNKS || !dims_ok(B, H, 1, D, E)) return LA_ERR_SHAPE;
+  if ((D != 64 && D != 128) || (E != 64 && E != 128)) return LA_ERR_UNSUPPORTED;
+  if ((R > 0 && !aligned16(states)) || !aligned16(out) || !aligned4(slopes) ||
+      (init_state && !aligned16(init_state)))
+    return LA_ERR_ALIGN;
+  la::CombineArgs a{};
+  for (int j = 0; j < R; ++j) {
+    if (chunk_tokens[j] < 0) return LA_ERR_SHAPE;
+    a.n[j] = chunk_tokens[j];
+  }
+  a.states = states;
+  a.init = init_state;
+  a.slopes = slopes;
+  a.out = out;
+  a.per_seq4 = static_cast<int64_t>(D) * E / 4;
+  a.total4 = static_cast<int64_t>(B) * H * a.per_seq4;
+  a.H = H;
+  a.R = R;
+  const int64_t blocks = (a.total4 + 255) / 256;
+  const int grid = static_cast<int>(blocks < 4 * 148 * 8 ? blocks : 4 * 148 * 8);
+  la::state_combine_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
 }
 
 const char* lightning_attn_last_cuda_error(void) { return t_last_cuda_error; }

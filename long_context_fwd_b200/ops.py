@@ -48,6 +48,8 @@ SIGNATURES = {
                                     _I, _I, _I, _P, _P, _P, _P, _P, _I, _P],
     "lightning_attn_decode_fused": [_P, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _I, _I, _I,
                                     _I, _P, _P, _P, _P, _P, _P],
+    "lightning_attn_state": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P],
+    "lightning_attn_state_combine": [_P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _P],
 }
 
 
@@ -313,6 +315,55 @@ def decode_fused(q, k, v, gate, state, slopes, norm_weight, eps: float = 1e-6, o
         slopes.data_ptr(), norm_weight.data_ptr(), float(eps), out.data_ptr(), B, H, D, E,
         *[ctypes.cast(a, ctypes.c_void_p) for a in arr], _stream_handle(stream))
     _check("lightning_attn_decode_fused", rc)
+    return out
+
+
+@_on_tensor_device
+def state(k, v, slopes, final_state=None, *, init_state=None, chunk: int = 0,
+          stream=None) -> torch.Tensor:
+    """The state after N tokens without the outputs: bf16 k [B,H,N,D], v [B,H,N,E]
+    -> fp32 [B,H,D,E] (from init_state, zero if None)."""
+    B, H, N, D = k.shape
+    E = v.shape[-1]
+    _need(k, "k", torch.bfloat16, (B, H, N, D))
+    _need(v, "v", torch.bfloat16, (B, H, N, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    if final_state is None:
+        final_state = torch.empty((B, H, D, E), dtype=torch.float32, device=k.device)
+    _need(final_state, "final_state", torch.float32, (B, H, D, E))
+    if init_state is not None:
+        _need(init_state, "init_state", torch.float32, (B, H, D, E))
+    rc = lib().lightning_attn_state(
+        k.data_ptr(), v.data_ptr(), slopes.data_ptr(),
+        None if init_state is None else init_state.data_ptr(), final_state.data_ptr(),
+        B, H, N, D, E, int(chunk), _stream_handle(stream))
+    _check("lightning_attn_state", rc)
+    return final_state
+
+
+@_on_tensor_device
+def state_combine(states, chunk_tokens, slopes, out=None, *, init_state=None,
+                  stream=None) -> torch.Tensor:
+    """The state after R consecutive chunks: fp32 states [R,B,H,D,E] (each chunk's
+    state from a zero initial state), chunk_tokens a sequence of R token counts
+    -> fp32 [B,H,D,E] (from init_state, zero if None)."""
+    R, B, H, D, E = states.shape
+    _need(states, "states", torch.float32, (R, B, H, D, E))
+    _need(slopes, "slopes", torch.float32, (H,))
+    counts = [int(x) for x in chunk_tokens]
+    if len(counts) != R:
+        raise ValueError(f"chunk_tokens must have {R} entries, got {len(counts)}")
+    if out is None:
+        out = torch.empty((B, H, D, E), dtype=torch.float32, device=states.device)
+    _need(out, "out", torch.float32, (B, H, D, E))
+    if init_state is not None:
+        _need(init_state, "init_state", torch.float32, (B, H, D, E))
+    arr = (ctypes.c_int * max(1, R))(*counts)
+    rc = lib().lightning_attn_state_combine(
+        states.data_ptr() if R else None, R, ctypes.cast(arr, ctypes.c_void_p),
+        slopes.data_ptr(), None if init_state is None else init_state.data_ptr(),
+        out.data_ptr(), B, H, D, E, _stream_handle(stream))
+    _check("lightning_attn_state_combine", rc)
     return out
 
 

@@ -101,7 +101,8 @@ def test_binding_runs_each_entry_on_its_tensors_device():
     # and refuses tensors spread over devices (checked with real devices on GPU
     # boxes; here the wrapper's pass-through for non-CUDA tensors)
     for name in ("fwd", "fwd_strided", "fwd_anticausal", "fwd_fused", "fwd_fused_ex", "bwd",
-                 "fwd_noalloc", "fwd_f32", "decode", "decode_fused", "fault_test_scan_stall"):
+                 "fwd_noalloc", "fwd_f32", "decode", "decode_fused", "state", "state_combine",
+                 "fault_test_scan_stall"):
         fn = getattr(ops, name)
         assert getattr(fn, "__wrapped__", None) is not None, name
     import torch
@@ -198,3 +199,30 @@ def test_fused_ex_and_decode_fused_validation(lib):
     assert g(*dargs(1e-6, (None,) * 5, D=96)) == LA_ERR_UNSUPPORTED
     assert g(*dargs(1e-6, (s2, s2, s2, C2(8 * 128, 132), s2))) == LA_ERR_ALIGN
     assert g(None, *dargs(1e-6, (None,) * 5)[1:]) == LA_ERR_NULL
+
+
+def test_state_and_combine_validation(lib):
+    f = lib.lightning_attn_state
+    assert f(FAKE, FAKE, FAKE, None, None, 1, 2, 8, 128, 128, 0, None) == LA_ERR_NULL  # final_state
+    assert f(None, FAKE, FAKE, None, FAKE, 1, 2, 8, 128, 128, 0, None) == LA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, None, FAKE, 1, 2, 0, 128, 128, 0, None) == LA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, None, FAKE, 1, 2, 8, 128, 128, 100, None) == LA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, None, FAKE, 1, 2, 8, 96, 128, 0, None) == LA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE + 8, FAKE, 1, 2, 8, 128, 128, 0, None) == LA_ERR_ALIGN
+    g = lib.lightning_attn_state_combine
+    C = ctypes.c_int * 3
+    n = C(100, 200, 300)
+    assert g(FAKE, 3, None, FAKE, None, FAKE, 1, 2, 128, 128, None) == LA_ERR_NULL
+    assert g(None, 3, ctypes.cast(n, ctypes.c_void_p), FAKE, None, FAKE, 1, 2, 128, 128,
+             None) == LA_ERR_NULL
+    assert g(FAKE, 257, ctypes.cast(n, ctypes.c_void_p), FAKE, None, FAKE, 1, 2, 128, 128,
+             None) == LA_ERR_SHAPE
+    assert g(FAKE, -1, ctypes.cast(n, ctypes.c_void_p), FAKE, None, FAKE, 1, 2, 128, 128,
+             None) == LA_ERR_SHAPE
+    bad = C(100, -1, 300)
+    assert g(FAKE, 3, ctypes.cast(bad, ctypes.c_void_p), FAKE, None, FAKE, 1, 2, 128, 128,
+             None) == LA_ERR_SHAPE
+    assert g(FAKE + 4, 3, ctypes.cast(n, ctypes.c_void_p), FAKE, None, FAKE, 1, 2, 128, 128,
+             None) == LA_ERR_ALIGN
+    assert g(FAKE, 3, ctypes.cast(n, ctypes.c_void_p), FAKE, None, FAKE, 1, 2, 128, 32,
+             None) == LA_ERR_UNSUPPORTED
