@@ -374,3 +374,27 @@ def test_bf16_large_initial_state_is_deterministic(B, H, N, chunk):
         if first is None:
             first = got
         assert np.array_equal(got, first)
+
+
+@pytest.mark.parametrize("B,H,N,mode", [(1, 64, 2500, 2), (2, 80, 1100, 1), (1, 3, 9000, 0)])
+def test_bf16_entering_items_are_deterministic(B, H, N, mode):
+    """Items that enter from a published state (split-scan shares, hand-over
+    continuations, chunks after the first) start with a large inter term:
+    repeated launches must be bitwise identical and match the oracle."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert ops.fwd_plan(B, H, N, 0, sms)[0]["mode"] == mode
+    q, k, v, _ = _bf16_case(B, H, N, [0.0] * H, seed=89 + mode)
+    sl = I.alibi_slopes(H)
+    sl[7::8] = 0.0
+    tq, tk, tv = (bf16_to_dev(x, DEV) for x in (q, k, v))
+    ts = f32_to_dev(sl, DEV)
+    first = None
+    for _ in range(4):
+        got = ops.fwd(tq, tk, tv, ts).cpu().numpy()
+        assert ops.device_status(reset=True) == 0
+        if first is None:
+            first = got
+            ref = oracle.recurrent(q, k, v, sl)
+            assert rel(got, ref) <= TOL_BF16
+            assert worst_head(got, ref) <= TOL_BF16
+        assert np.array_equal(got, first)
