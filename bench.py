@@ -515,8 +515,9 @@ def bench_decode(args, dist, dev, fused: bool = False):
 
 def bench_backward(args, dist, w, dev):
     """The backward pass (dq, dk, dv from dout) on the prefill workload's shapes:
-    three launches of the tensor-core kernel per step (dq causal, dk and dv
-    anti-causal), inputs resident on the device."""
+    launches of the tensor-core kernel per step: dq causal, then dk and dv
+    anti-causal (one paired launch when D == E, else one each), inputs
+    resident on the device."""
     import torch
     from long_context_fwd_b200 import inputs as I
     from long_context_fwd_b200 import ops
@@ -550,11 +551,18 @@ def bench_backward(args, dist, w, dev):
     del q, k, v, dout, dq, dk, dv
     torch.cuda.empty_cache()
     units = w.B * w.H * w.N
-    # three launches, each reading three bf16 operands and writing fp32
-    moved = units * (2 * (2 * w.E + w.D) + 4 * w.D + 2 * (2 * w.D + w.E) + 4 * w.D +
-                     2 * (2 * w.D + w.E) + 4 * w.E)
+    # streamed operands: the dq launch reads dout, v, k and writes dq; the
+    # paired dk/dv launch reads q, k, v, dout (each q and dout tile from DRAM
+    # once when the second role's read hits L2) and writes dk, dv; unpaired,
+    # dk and dv each read three operands
+    paired = w.D == w.E
+    moved = units * (2 * (2 * w.E + w.D) + 4 * w.D)
+    if paired:
+        moved += units * (2 * (2 * w.D + 2 * w.E) + 4 * w.D + 4 * w.E)
+    else:
+        moved += units * (2 * (2 * w.D + w.E) + 4 * w.D + 2 * (2 * w.D + w.E) + 4 * w.E)
     return {"ms": ms, "steps": steps, "window": (t_host0, t_host1), "status": status,
-            "launches": 3, "bytes_moved": moved}
+            "launches": 2 if paired else 3, "bytes_moved": moved}
 
 
 def bench_fused(args, dist, w, dev):

@@ -224,11 +224,14 @@ int lightning_attn_fwd_anticausal(const void* q, const void* k, const void* v, c
  *   dv_s = sum_{t >= s} g^(t-s) (q_t . k_s) dout_t      dv [B][H][N][E]
  * (g = exp(-lambda_h); zero initial state; the slopes are not differentiated).
  * dq is the causal operator applied to (dout, v, k); dk and dv are the
- * anti-causal operator applied to (v, dout, q) and (k, q, dout): three
- * launches of the tensor-core kernel on `stream`.  bf16 inputs as for the
- * forward pass, D, E in {64, 128}; dq, dk, dv 16-byte aligned and not
- * overlapping the inputs or each other (not checked).  Errors as
- * lightning_attn_fwd (the first failing launch's code).
+ * anti-causal operator applied to (v, dout, q) and (k, q, dout).  With D == E
+ * dk and dv share one launch whose CTAs alternate between them on the same
+ * work items, so q and dout are streamed from memory about once for both (two
+ * launches of the tensor-core kernel on `stream`); otherwise three launches.
+ * bf16 inputs as for the forward pass, D, E in {64, 128}; dq, dk, dv 16-byte
+ * aligned and not overlapping the inputs or each other (not checked).  Errors
+ * as lightning_attn_fwd: LA_ERR_NULL or LA_ERR_ALIGN before any launch, else
+ * the first failing launch's code.
  */
 int lightning_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
                        const float* slopes, float* dq, float* dk, float* dv, int B, int H, int N,

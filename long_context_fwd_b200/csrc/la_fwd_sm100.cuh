@@ -130,10 +130,22 @@ __device__ __forceinline__ void trace_event(int ev, uint32_t idx) {
 #define LA_TRACE_EVENT(ev, idx) ((void)0)
 #endif
 
+// A paired launch runs two operators on alternate CTAs: the schedule sees a
+// grid of half the CTAs, and each role has its own scratch and output.
+__device__ __forceinline__ int cta_role(const Params& p) {
+  return p.paired ? static_cast<int>(blockIdx.x & 1u) : 0;
+}
+__device__ __forceinline__ int vgrid(const Params& p) {
+  return static_cast<int>(gridDim.x >> (p.paired ? 1 : 0));
+}
+__device__ __forceinline__ int vcta(const Params& p) {
+  return static_cast<int>(blockIdx.x >> (p.paired ? 1 : 0));
+}
+
 // Work item for work index w on this CTA.
 __device__ __forceinline__ bool get_item(const Params& p, const volatile uint32_t* m, int w,
                                          Item& it) {
-  return get_item(p, static_cast<int>(gridDim.x), static_cast<int>(blockIdx.x), m, w, it);
+  return get_item(p, vgrid(p), vcta(p), m, w, it);
 }
 
 __device__ __forceinline__ void st_release_gpu(unsigned long long* ptr, unsigned long long v) {
@@ -316,8 +328,8 @@ __device__ __forceinline__ bool gsync(const Ctx& c, const Params& p, int id, uin
 // for chunked runs, a static stride otherwise (n counts this CTA's items).
 __device__ __forceinline__ int next_work(const Params& p, int& n) {
   if (p.mode != MODE_TICKETS) return n++;
-  if (p.nchunks > 1) return p.ticket_base + atomicAdd(p.ticket, 1);
-  return blockIdx.x + gridDim.x * n++;
+  if (p.nchunks > 1) return p.ticket_base + atomicAdd(cta_role(p) ? p.ticket1 : p.ticket, 1);
+  return vcta(p) + vgrid(p) * n++;
 }
 
 // Coordinates (beyond the column) of a tile of tokens [row, row + 128) of
@@ -804,6 +816,11 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
   const bool leader = (t == 0);
   const uint64_t pol_out = policy_evict_first();
   uint32_t v_it = 0, w_it = 0, gb = 0, agg_n = 0, ys_n = 0;
+  // this CTA's scratch and plain-store output (the second role's in a paired launch)
+  const bool role1 = cta_role(p) != 0;
+  float* const prefix = role1 ? p.prefix1 : p.prefix;
+  unsigned long long* const flags = role1 ? p.flags1 : p.flags;
+  float* const out = role1 ? p.out1 : p.out;
   // kvb row address of column quarter q (32 columns): plane q / 2, chunks 4 (q % 2)..
   auto kvb_row = [&](uint32_t q) { return c.sbase + OFF_KVB + (q >> 1) * PLANE + r * 128u; };
 
@@ -826,7 +843,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     // split scan: the entering state chains the published local states of the
     // stream pieces [s F, X) (X = stream position of this item's first block)
     const bool chain = it.enter && p.mode == MODE_SPLIT_SCAN;
-    const int64_t G = gridDim.x;
+    const int64_t G = vgrid(p);
     const int64_t x_lo = static_cast<int64_t>(it.seq) * p.F;
     const int64_t x_hi = x_lo + it.t0 / BLK;
     if (it.enter) {
@@ -838,7 +855,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         int slot = chain ? s1_slot(p, G, x) : it.enter_slot;
         uint32_t n = 0;
         for (;;) {
-          if (ld_acquire_gpu(p.flags + slot) == it.enter_val) {
+          if (ld_acquire_gpu(flags + slot) == it.enter_val) {
             if (!chain) break;
             const int64_t y = s1_next(p, G, x);
             if (n == CHAIN_MAX) {  // excluded by the host's plan; no wrong result
@@ -861,7 +878,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         c.misc[18] = n;
       }
       if (!gsync(c, p, B_YSYNC, ys_n)) break;
-      if (!chain) scan_src = p.prefix + static_cast<int64_t>(it.enter_slot) * (HD * HD);
+      if (!chain) scan_src = prefix + static_cast<int64_t>(it.enter_slot) * (HD * HD);
     }
     // the caller's initial state enters at block 0 of a sequence (or through
     // the chain); never into a local state -- except in the state pass, where
@@ -875,7 +892,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     {
       const float gL = expf(-lam * static_cast<float>(it.Lc));
       const float g0 = expf(-lam * static_cast<float>(min(BLK, it.Lc)));
-      float* pub = p.prefix + static_cast<int64_t>(it.pub_slot) * (HD * HD);
+      float* pub = prefix + static_cast<int64_t>(it.pub_slot) * (HD * HD);
 #pragma unroll 1
       for (uint32_t q = 0; q < 4; ++q) {
         uint32_t prev[32];
@@ -896,7 +913,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
 #pragma unroll 1
           for (int j = 0; j < n; ++j) {
             uint32_t part[32];
-            ld_scan32(p.prefix + static_cast<int64_t>(c.chain[2 * j]) * (HD * HD), r, q >> 1, q & 1u, part);
+            ld_scan32(prefix + static_cast<int64_t>(c.chain[2 * j]) * (HD * HD), r, q >> 1, q & 1u, part);
             const float w = expf(-lam * static_cast<float>(static_cast<int>(c.chain[2 * j + 1]) * BLK));
 #pragma unroll
             for (int i = 0; i < 32; ++i)
@@ -931,7 +948,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
       if (!gsync(c, p, B_YSYNC, ys_n)) break;
       if (leader) {
         __threadfence();
-        st_release_gpu(p.flags + it.pub_slot, it.pub_val);
+        st_release_gpu(flags + it.pub_slot, it.pub_val);
       }
     }
     if (leader) LA_TRACE_EVENT(19, w_it);
@@ -947,8 +964,8 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     float* const fin_dst = it.last && p.final_state && row_in
                                ? p.final_state + static_cast<int64_t>(it.seq) * state_elems + row_off
                                : nullptr;
-    float* const pub_dst = it.publish ? p.prefix + static_cast<int64_t>(it.pub_slot) * (HD * HD) : nullptr;
-    unsigned long long* const pub_flag = it.publish ? p.flags + it.pub_slot : nullptr;
+    float* const pub_dst = it.publish ? prefix + static_cast<int64_t>(it.pub_slot) * (HD * HD) : nullptr;
+    unsigned long long* const pub_flag = it.publish ? flags + it.pub_slot : nullptr;
     const unsigned long long pub_val = it.pub_val;
     bool ok = true;
     for (int n = 0; n < it.nb && ok; ++n) {
@@ -1007,7 +1024,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         // negative row, where a TMA store may not start: plain stores of the
         // rows that exist, straight from TMEM.  The V slot is not needed.
         const int tok = row + static_cast<int>(r);
-        float* dst = tok >= 0 ? p.out + (it.seq / p.H) * p.ostride[0] + (it.seq % p.H) * p.ostride[1] +
+        float* dst = tok >= 0 ? out + (it.seq / p.H) * p.ostride[0] + (it.seq % p.H) * p.ostride[1] +
                                      static_cast<int64_t>(tok) * p.ostride[2]
                               : nullptr;
 #pragma unroll 1
@@ -1170,6 +1187,8 @@ template <int RANK, bool REV, bool FUSED>
 __global__ void __launch_bounds__(THREADS, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                    const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap tk1,
+                    const __grid_constant__ CUtensorMap tv1, const __grid_constant__ CUtensorMap to1,
                     const Params p) {
   extern __shared__ uint8_t smem_raw[];
   Ctx c;
@@ -1211,7 +1230,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&c.bar[B_YSYNC], Y_WARPS);
     mbar_init(&c.bar[B_DRAIN], 1);
     c.misc[3] = 0;
-    if (!setup_split(p, static_cast<int>(gridDim.x), static_cast<int>(blockIdx.x), c.misc)) {
+    if (!setup_split(p, vgrid(p), vcta(p), c.misc)) {
       c.misc[4] = 0;  // cannot happen (see split_scan_setup); no work rather than wrong work
       atomicOr(p.status, 4);
     }
@@ -1221,11 +1240,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(const_cast<uint32_t*>(&c.misc[0]), 512);
     tmem_relinquish();
   }
+  const bool role1 = cta_role(p) != 0;
+  const CUtensorMap* const mq = role1 ? &tq1 : &tq;
+  const CUtensorMap* const mk = role1 ? &tk1 : &tk;
+  const CUtensorMap* const mv = role1 ? &tv1 : &tv;
+  const CUtensorMap* const mo = role1 ? &to1 : &to;
   if (warp == PRODUCER_WARP && lane_id() == 0) {
-    prefetch_tmap(&tq);
-    prefetch_tmap(&tk);
-    prefetch_tmap(&tv);
-    prefetch_tmap(&to);
+    prefetch_tmap(mq);
+    prefetch_tmap(mk);
+    prefetch_tmap(mv);
+    prefetch_tmap(mo);
   }
   tc_fence_before();
   __syncthreads();
@@ -1233,14 +1257,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   c.tmem = c.misc[0];
 
   if (warp == PRODUCER_WARP) {
-    if (lane_id() == 0) producer<RANK, REV>(c, p, &tq, &tk, &tv);
+    if (lane_id() == 0) producer<RANK, REV>(c, p, mq, mk, mv);
   } else if (warp == MMA_WARP) {
     if (lane_id() == 0) mma_issuer<FUSED>(c, p);
     __syncwarp();
   } else if (warp < Y_WARP0) {
     group_x<REV, FUSED>(c, p);
   } else {
-    group_y<RANK, REV, FUSED>(c, p, &to);
+    group_y<RANK, REV, FUSED>(c, p, mo);
   }
 
   tc_fence_before();

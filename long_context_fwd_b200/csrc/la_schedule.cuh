@@ -46,6 +46,14 @@ struct Params {
   const float* norm_w;        // fused layer: RMSNorm weight [H][E]
   float eps;                  // fused layer: RMSNorm epsilon
   unsigned long long wait_limit_ns;
+  // Two operators in one launch (paired = 1): CTA 2j + r computes role r of
+  // virtual CTA j (role 1 takes the second set of tensor maps and these
+  // pointers), so both roles of a pair read shared operands close in time.
+  int paired;
+  int* ticket1;
+  unsigned long long* flags1;
+  float* prefix1;
+  float* out1;
 };
 
 // How sequences become work items (chosen on the host):

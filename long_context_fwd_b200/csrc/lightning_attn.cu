@@ -69,8 +69,11 @@ int sm_count() {
 // every thread of the process (lightning_attn_set_cta_limit).
 std::atomic<int> g_cta_limit{0};
 
+// The prefill kernel takes two sets of q, k, v, out tensor maps: the second is
+// role 1's in a paired launch (a copy of the first otherwise).
 using FwdKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                           const CUtensorMap, const la::fwd::Params);
+                           const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                           const CUtensorMap, const CUtensorMap, const la::fwd::Params);
 
 FwdKernel pick_fwd_kernel(int rank, bool rev, bool fused) {
   using la::fwd::fwd_bf16_kernel;
@@ -374,9 +377,11 @@ bool build_maps(const void* q, const void* k, const void* v, const void* out, in
 // launch) instead of leaving a waiting CTA on an SM that a CTA it waits for
 // needs.  The chunk scan hands work out by ticket in order and needs no such
 // guarantee.
+// role1: the second role's four maps (q, k, v, out) of a paired launch, or null.
 int launch_fwd(FwdKernel kern, int grid, bool cooperative, cudaStream_t stream,
                const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-               const CUtensorMap& to, const la::fwd::Params& p) {
+               const CUtensorMap& to, const la::fwd::Params& p,
+               const CUtensorMap* role1 = nullptr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(la::fwd::THREADS);
@@ -387,7 +392,9 @@ int launch_fwd(FwdKernel kern, int grid, bool cooperative, cudaStream_t stream,
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = cooperative ? 1 : 0;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, p);
+  const cudaError_t e =
+      role1 ? cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, role1[0], role1[1], role1[2], role1[3], p)
+            : cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, tq, tk, tv, to, p);
   if (e != cudaSuccess) return cuda_fail(e);
   return launch_status();
 }
@@ -682,13 +689,92 @@ int lightning_attn_fwd_anticausal(const void* q, const void* k, const void* v, c
                        stream, nullptr, /*reverse=*/true);
 }
 
+// dk and dv in one launch.  Both are anti-causal operators that read q and
+// dout (dk on (v, dout, q), dv on (k, q, dout)), so CTA 2j computes dk and CTA
+// 2j + 1 dv of the same work items, planned for half the CTAs: the two CTAs
+// of a pair stream the same q and dout tiles at about the same time, and the
+// second read of each comes from L2.  Each role has its own scratch (ticket,
+// flags, hand-over states).  Needs D == E and at least two CTAs; *applies is
+// false (and nothing is launched) otherwise.
+int bwd_pair_impl(const void* q, const void* k, const void* v, const void* dout,
+                  const float* slopes, float* dk, float* dv, int B, int H, int N, int D, int E,
+                  cudaStream_t stream, bool* applies) {
+  *applies = false;
+  if (D != E) return LA_OK;
+  const FwdKernel kern = pick_fwd_kernel(3, true, false);
+  int ctas = 0;
+  int rc = prepare_fwd_kernel(kern, &ctas);
+  if (rc != LA_OK) return rc;
+  if (ctas < 2) return LA_OK;
+  *applies = true;
+  const int nseq = B * H;
+  la::fwd::Params p{};
+  CUtensorMap m0[4], m1[4];
+  int rank0 = 0, rank1 = 0;
+  const Strides st = contiguous_strides(H, N, D, E);
+  if (!build_maps(v, dout, q, dk, B, H, N, D, E, st, &m0[0], &m0[1], &m0[2], &m0[3], p, &rank0) ||
+      !build_maps(k, q, dout, dv, B, H, N, D, E, st, &m1[0], &m1[1], &m1[2], &m1[3], p, &rank1) ||
+      rank0 != 3 || rank1 != 3)
+    return LA_ERR_CUDA;
+  const Plan pl = make_plan(nseq, N, ctas / 2, 0);
+  if (pl.total >= (1ll << 31)) return LA_ERR_SHAPE;
+  p.out = dk;
+  p.out1 = dv;
+  for (int j = 0; j < 3; ++j) p.ostride[j] = st.s[3][j];
+  p.slopes = slopes;
+  p.status = status_word();
+  if (!p.status) return LA_ERR_CUDA;
+  p.H = H;
+  p.N = N;
+  apply_plan(pl, nseq, p);
+  p.wait_limit_ns = kWaitLimitNs;
+  p.tag = launch_tag();
+  p.paired = 1;
+  void* scratch = nullptr;
+  if (pl.bytes) {  // role 0's scratch, then role 1's (pl.bytes is a multiple of 256)
+    cudaError_t e = cudaMallocAsync(&scratch, 2 * pl.bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (needs_zeroed_ctrl(pl, stream)) {
+      e = cudaMemsetAsync(scratch, 0, pl.ctrl, stream);
+      if (e == cudaSuccess)
+        e = cudaMemsetAsync(static_cast<char*>(scratch) + pl.bytes, 0, pl.ctrl, stream);
+      if (e != cudaSuccess) {
+        cudaFreeAsync(scratch, stream);
+        return cuda_fail(e);
+      }
+    }
+    la::fwd::Params p1{};
+    set_scratch(pl, static_cast<char*>(scratch) + pl.bytes, p1);
+    set_scratch(pl, scratch, p);
+    p.ticket1 = p1.ticket;
+    p.flags1 = p1.flags;
+    p.prefix1 = p1.prefix;
+  }
+  rc = launch_fwd(kern, 2 * pl.grid, pl.mode != la::fwd::MODE_TICKETS, stream, m0[0], m0[1],
+                  m0[2], m0[3], p, m1);
+  if (scratch) {
+    const cudaError_t e = cudaFreeAsync(scratch, stream);
+    if (e != cudaSuccess && rc == LA_OK) rc = cuda_fail(e);
+  }
+  return rc;
+}
+
 int lightning_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
                        const float* slopes, float* dq, float* dk, float* dv, int B, int H, int N,
                        int D, int E, void* stream) {
-  if (!dout || !dq || !dk || !dv) return LA_ERR_NULL;
+  if (!q || !k || !v || !dout || !slopes || !dq || !dk || !dv) return LA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned4(slopes))
+    return LA_ERR_ALIGN;
   // dq_t = sum_{s<=t} g^(t-s) (dout_t . v_s) k_s: the causal operator on (dout, v, k)
   int rc = fwd_bf16_impl(dout, v, k, slopes, nullptr, nullptr, dq, B, H, N, E, D, 0, stream);
   if (rc != LA_OK) return rc;
+  // dk and dv: one paired launch when D == E (the dq launch has checked the
+  // shapes, and the pointers are checked above)
+  bool paired = false;
+  rc = bwd_pair_impl(q, k, v, dout, slopes, dk, dv, B, H, N, D, E,
+                     static_cast<cudaStream_t>(stream), &paired);
+  if (paired || rc != LA_OK) return rc;
   // dk_s = sum_{t>=s} g^(t-s) (v_s . dout_t) q_t: the anti-causal operator on (v, dout, q)
   rc = fwd_bf16_impl(v, dout, q, slopes, nullptr, nullptr, dk, B, H, N, E, D, 0, stream, nullptr,
                      true);

@@ -1,8 +1,10 @@
 """GPU parity of the anti-causal prefill and the backward pass against the oracle.
 
 lightning_attn_fwd_anticausal runs the tensor-core kernel in reversed time;
-lightning_attn_bwd composes three launches (dq causal on (dout, v, k); dk, dv
-anti-causal on (v, dout, q) and (k, q, dout)).  Both are compared element by
+lightning_attn_bwd composes dq (causal on (dout, v, k)) with dk and dv
+(anti-causal on (v, dout, q) and (k, q, dout)), the last two in one paired
+launch when D == E (alternate CTAs, each role planned for half the grid) and
+in two launches otherwise.  Both are compared element by
 element with the float64 oracle (its anti-causal sum and its gradients of
 L = sum dout . o, pinned in tests/test_oracle_backward.py) on the same seeded
 bf16 inputs, across the kernel's work splits (whole sequences, explicit
@@ -111,3 +113,27 @@ def test_backward_adjoint_identity_on_device():
     for x, dx in ((dq_, dq), (dk_, dk), (dv_, dv)):
         lx = (x.double() * dx.double()).sum(dim=(2, 3))
         assert torch.allclose(lx, L, rtol=2e-2, atol=1e-3 * float(L.abs().max()))
+
+
+@pytest.mark.parametrize("B,H,N,mode", [
+    (2, 80, 600, 1),    # hand-over
+    (1, 64, 2000, 2),   # split scan
+    (1, 4, 3000, 0),    # chunk scan: each role draws its own tickets
+    (1, 2, 1000, 0),    # whole sequences
+    (1, 1, 1, 0),       # one token
+])
+def test_backward_paired_launch_every_split(B, H, N, mode):
+    """dk and dv from the paired launch, whose roles each plan for half the
+    CTAs, in every work split of that plan."""
+    sms = torch.cuda.get_device_properties(DEV).multi_processor_count
+    assert ops.fwd_plan(B, H, N, 0, sms // 2)[0]["mode"] == mode
+    q, k, v, g, sl = _case(B, H, N, 128, 128, seed=300 + H + N % 29)
+    dq, dk, dv = ops.bwd(*(bf16_to_dev(x, DEV) for x in (q, k, v, g)), f32_to_dev(sl, DEV))
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0
+    refs = oracle.backward(q, k, v, g, sl)
+    for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), refs):
+        a = got.cpu().numpy()
+        assert np.isfinite(a).all(), name
+        assert rel(a, ref) <= TOL_BF16, name
+        assert worst_head(a, ref) <= TOL_BF16, name

@@ -108,3 +108,24 @@ def test_other_entries_on_a_capped_grid(entry, cta_limit):
     got = got.float().cpu().numpy()
     assert rel(got, ref) <= TOL_BF16
     assert worst_head(got, ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("ctas", [1, 3, 37])
+def test_backward_on_capped_grid(ctas, cta_limit):
+    """The backward pass on grids of 1 CTA (dk and dv then take a launch each),
+    3 CTAs (one pair: dk and dv side by side) and 37 (18 pairs)."""
+    B, H, N = 1, 64, 1300
+    cta_limit(ctas)
+    w = I.Workload("capbwd", B, H, N, 128, 128, "bf16", index=880 + ctas)
+    q, k, v = I.prefill_inputs(w)
+    g = I.f32_to_bf16_bits(np.random.default_rng(ctas).standard_normal((B, H, N, 128))
+                           .astype(np.float32))
+    sl = I.alibi_slopes(H)
+    dq, dk, dv = ops.bwd(*(bf16_to_dev(x, DEV) for x in (q, k, v, g)), f32_to_dev(sl, DEV))
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0
+    refs = oracle.backward(q, k, v, g, sl)
+    for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), refs):
+        a = got.cpu().numpy()
+        assert rel(a, ref) <= TOL_BF16, name
+        assert worst_head(a, ref) <= TOL_BF16, name
