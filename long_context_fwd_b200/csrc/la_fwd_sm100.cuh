@@ -847,35 +847,43 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     const int64_t x_lo = static_cast<int64_t>(it.seq) * p.F;
     const int64_t x_hi = x_lo + it.t0 / BLK;
     if (it.enter) {
-      if (leader) {
-        // wait for each piece in turn and note it in the chain list
-        const uint64_t t0 = globaltimer_ns();
-        uint32_t spins = 0;
-        int64_t x = x_lo;
-        int slot = chain ? s1_slot(p, G, x) : it.enter_slot;
-        uint32_t n = 0;
-        for (;;) {
-          if (ld_acquire_gpu(flags + slot) == it.enter_val) {
-            if (!chain) break;
-            const int64_t y = s1_next(p, G, x);
-            if (n == CHAIN_MAX) {  // excluded by the host's plan; no wrong result
+      if (t < 32) {  // the group's first warp waits
+        // The chain's pieces follow from the plan alone: lane 0 lists them
+        // (slot, distance to X), then every lane waits for one piece's flag,
+        // so the pieces' publication latencies overlap instead of adding up.
+        if (chain && t == 0) {
+          uint32_t m = 0;
+          for (int64_t x = x_lo; x < x_hi;) {
+            if (m == CHAIN_MAX) {  // excluded by the host's plan; no wrong result
               fail(c, p, 4);
+              m = 0;
               break;
             }
-            c.chain[2 * n] = static_cast<uint32_t>(slot);
-            c.chain[2 * n + 1] = static_cast<uint32_t>(x_hi - y);
-            ++n;
+            const int64_t y = s1_next(p, G, x);
+            c.chain[2 * m] = static_cast<uint32_t>(s1_slot(p, G, x));
+            c.chain[2 * m + 1] = static_cast<uint32_t>(x_hi - y);
+            ++m;
             x = y;
-            if (x >= x_hi) break;
-            slot = s1_slot(p, G, x);
-            continue;
           }
-          if ((++spins & 15u) == 0 && (aborted(c) || globaltimer_ns() - t0 > p.wait_limit_ns)) {
-            fail(c, p, 2);
+          c.misc[18] = m;
+        }
+        __syncwarp();
+        const uint32_t n = chain ? c.misc[18] : 1u;
+        const unsigned long long* f =
+            t < n ? flags + (chain ? static_cast<int>(c.chain[2 * t]) : it.enter_slot) : nullptr;
+        bool seen = f == nullptr;
+        const uint64_t t0 = globaltimer_ns();
+        uint32_t spins = 0;
+        for (;;) {
+          if (!seen) seen = ld_acquire_gpu(f) == it.enter_val;
+          if (__all_sync(0xffffffffu, seen)) break;
+          // spins is the same in every lane, so the lanes decide together
+          if ((++spins & 15u) == 0 &&
+              __any_sync(0xffffffffu, aborted(c) || globaltimer_ns() - t0 > p.wait_limit_ns)) {
+            if (t == 0) fail(c, p, 2);
             break;
           }
         }
-        c.misc[18] = n;
       }
       if (!gsync(c, p, B_YSYNC, ys_n)) break;
       if (!chain) scan_src = prefix + static_cast<int64_t>(it.enter_slot) * (HD * HD);

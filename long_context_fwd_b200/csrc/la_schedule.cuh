@@ -253,9 +253,10 @@ LA_HD bool split_scan_item(const Params& p, int i, const volatile uint32_t* m, i
       if (r1 <= r0) return false;
       const int sa = r0 / F, sb = (r1 - 1) / F;
       if (k2 > sb - sa) return false;
-      // a first piece that needs an entering state goes last (more time for
-      // the local-state pass to finish)
-      if (r0 > sa * F) k2 = k2 == sb - sa ? 0 : k2 + 1;
+      // in stream order: a first piece that needs an entering state starts
+      // right after this CTA's local-state pass, when the pieces it chains
+      // have just been published (still in L2) -- later, behind a stream of
+      // output blocks, their loads took several times longer
       seq = sa + k2;
       blk0 = la_max(r0, seq * F) - seq * F;
       blk1 = la_min(r1, (seq + 1) * F) - seq * F;
