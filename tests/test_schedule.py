@@ -209,11 +209,13 @@ def _check_split_scan(B, H, N, sms, info, items):
                 # the kernel notes the chain in a 32-entry shared-memory list
                 assert len(links) <= 32
         kinds = [it["kind"] for it in its]
-        # local-state items first, then outputs (the entering one last)
+        # local-state items first, then outputs in stream order (so only the
+        # first output item can enter a sequence part-way)
         first_out = kinds.index(0) if 0 in kinds else len(kinds)
         assert all(k == 1 for k in kinds[:first_out])
         outs = [it for it in its if it["kind"] == 0]
-        assert all(not it["flags"] & ENTER for it in outs[:-1])
+        assert all(not it["flags"] & ENTER for it in outs[1:])
+        assert all((a["seq"], a["a"]) < (b["seq"], b["a"]) for a, b in zip(outs, outs[1:]))
     # both passes are balanced
     P = nseq * F
     for cta, its in by.items():
