@@ -185,9 +185,6 @@ __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t x, float f) {
   return pack_bf16x2(bf16lo_to_f32(x) * f, bf16hi_to_f32(x) * f);
 }
 
-// Multiplies the 64 bf16 of one 128-byte swizzled row by f, in place.  All 8
-// loads are issued before any store; the physical chunk order (c ^ row) keeps
-// 8 consecutive rows on distinct banks.
 // sigmoid(x) = (1 + tanh(x / 2)) / 2 from the hardware tanh (tanh.approx.f32,
 // one MUFU operation per element): the fused layer's gate.
 __device__ __forceinline__ float tanh_hw(float x) {
@@ -225,6 +222,9 @@ __device__ __forceinline__ void silu_row(uint32_t rowaddr, uint32_t row, float f
   for (uint32_t c = 0; c < 8; ++c) sts128(rowaddr + ((c ^ (row & 7u)) << 4), x[c]);
 }
 
+// Multiplies the 64 bf16 of one 128-byte swizzled row by f, in place.  All 8
+// loads are issued before any store; the physical chunk order (c ^ row) keeps
+// 8 consecutive rows on distinct banks.
 __device__ __forceinline__ void scale_row(uint32_t rowaddr, uint32_t row, float f) {
   uint4 x[8];
 #pragma unroll
