@@ -615,13 +615,13 @@ def cpu_baseline(w, seconds: float):
 
     sl = I.slopes_for(w)
 
-    def run(b, n):
+    def run(b, n, threads=0):
         arrs = [I.head_inputs(w, b, h, 0, n) for h in range(w.H)]
         q = np.stack([a[0] for a in arrs])[None]
         k = np.stack([a[1] for a in arrs])[None]
         v = np.stack([a[2] for a in arrs])[None]
         t0 = time.time()
-        oracle.recurrent(q, k, v, sl)
+        oracle.recurrent(q, k, v, sl, threads=threads)
         return time.time() - t0
 
     n = 128
@@ -632,9 +632,14 @@ def cpu_baseline(w, seconds: float):
         while rows < w.B and total * (rows + 1) / rows < seconds:
             total += run(rows, n)
             rows += 1
+    # one core on a shorter prefix of batch row 0 (about a fifth of the budget)
+    n1 = int(min(w.N, max(16, n * (seconds / 5) / max(total / rows, 1e-3) / oracle.max_threads())))
+    t1 = run(0, n1, threads=1)
     return {"value": rows * n / total, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
             "sample": f"float64 recurrence, batch rows 0..{rows - 1} of {w.B}, all {w.H} heads, "
-                      f"first {n} of {w.N} tokens ({total:.1f} s)"}
+                      f"first {n} of {w.N} tokens ({total:.1f} s)",
+            "single_core": {"value": n1 / t1, "unit": "tokens/s",
+                            "sample": f"batch row 0, all {w.H} heads, first {n1} tokens ({t1:.1f} s)"}}
 
 
 def job_throughput(world: int, units_per_rank: int, ms_per_step_max: float) -> float:

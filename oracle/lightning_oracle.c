@@ -92,11 +92,15 @@ static int bad_args(const void* q, const void* k, const void* v, const float* sl
   return 0;
 }
 
-static void set_threads(int nthreads) {
+/* Threads for one call: nthreads if positive, else the OpenMP default.  Passed
+ * to each parallel loop (num_threads), so one call's choice never changes the
+ * next call's default. */
+static int pick_threads(int nthreads) {
 #ifdef _OPENMP
-  if (nthreads > 0) omp_set_num_threads(nthreads);
+  return nthreads > 0 ? nthreads : omp_get_max_threads();
 #else
   (void)nthreads;
+  return 1;
 #endif
 }
 
@@ -106,9 +110,9 @@ int la_oracle_masked(const void* q, const void* k, const void* v, int dtype,
                      int64_t B, int64_t H, int64_t N, int64_t D, int64_t E, int nthreads) {
   int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
   if (rc) return rc;
-  set_threads(nthreads);
+  const int nt = pick_threads(nthreads);
   int64_t BH = B * H;
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
   for (int64_t bh = 0; bh < BH; ++bh) {
     double lam = (double)slopes[bh % H];
     double* Q = (double*)malloc(sizeof(double) * (size_t)(N * D + 1));
@@ -144,9 +148,9 @@ int la_oracle_recurrent(const void* q, const void* k, const void* v, int dtype,
                         int64_t B, int64_t H, int64_t N, int64_t D, int64_t E, int nthreads) {
   int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
   if (rc) return rc;
-  set_threads(nthreads);
+  const int nt = pick_threads(nthreads);
   int64_t BH = B * H;
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
   for (int64_t bh = 0; bh < BH; ++bh) {
     double gamma = exp(-(double)slopes[bh % H]);
     double* S = (double*)calloc((size_t)(D * E), sizeof(double));
@@ -187,9 +191,9 @@ int la_oracle_recurrent_sampled(const void* q, const void* k, const void* v, int
   if (npos < 0 || (npos > 0 && !pos)) return 1;
   for (int64_t p = 0; p < npos; ++p)
     if (pos[p] < 0 || pos[p] >= N) return 2;
-  set_threads(nthreads);
+  const int nt = pick_threads(nthreads);
   int64_t BH = B * H;
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
   for (int64_t bh = 0; bh < BH; ++bh) {
     double gamma = exp(-(double)slopes[bh % H]);
     double* S = (double*)calloc((size_t)(D * E), sizeof(double));
@@ -238,9 +242,9 @@ int la_oracle_blocked(const void* q, const void* k, const void* v, int dtype,
   int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
   if (rc) return rc;
   if (blk < 1) return 2;
-  set_threads(nthreads);
+  const int nt = pick_threads(nthreads);
   int64_t BH = B * H;
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
   for (int64_t bh = 0; bh < BH; ++bh) {
     double lam = (double)slopes[bh % H];
     double* S = (double*)calloc((size_t)(D * E), sizeof(double));
@@ -301,9 +305,9 @@ int la_oracle_decode_step(const void* q, const void* k, const void* v, int dtype
   int rc = bad_args(q, k, v, slopes, out, B, H, 1, D, E);
   if (rc) return rc;
   if (!state) return 1;
-  set_threads(nthreads);
+  const int nt = pick_threads(nthreads);
   int64_t BH = B * H;
-#pragma omp parallel for schedule(dynamic, 16)
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 16)
   for (int64_t bh = 0; bh < BH; ++bh) {
     double gamma = exp(-(double)slopes[bh % H]);
     double* S = state + bh * D * E;
@@ -327,9 +331,9 @@ int la_oracle_masked_anticausal(const void* q, const void* k, const void* v, int
                                 int64_t D, int64_t E, int nthreads) {
   int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
   if (rc) return rc;
-  set_threads(nthreads);
+  const int nt = pick_threads(nthreads);
   int64_t BH = B * H;
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
   for (int64_t bh = 0; bh < BH; ++bh) {
     double lam = (double)slopes[bh % H];
     double* Q = (double*)malloc(sizeof(double) * (size_t)(N * D + 1));
@@ -366,9 +370,9 @@ int la_oracle_recurrent_anticausal(const void* q, const void* k, const void* v, 
                                    int64_t E, int nthreads) {
   int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
   if (rc) return rc;
-  set_threads(nthreads);
+  const int nt = pick_threads(nthreads);
   int64_t BH = B * H;
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
   for (int64_t bh = 0; bh < BH; ++bh) {
     double gamma = exp(-(double)slopes[bh % H]);
     double* S = (double*)calloc((size_t)(D * E), sizeof(double));
@@ -408,9 +412,9 @@ int la_oracle_backward_masked(const void* q, const void* k, const void* v, const
   int rc = bad_args(q, k, v, slopes, dq, B, H, N, D, E);
   if (rc) return rc;
   if (bad_grads(dout, dq, dk, dv)) return 1;
-  set_threads(nthreads);
+  const int nt = pick_threads(nthreads);
   int64_t BH = B * H;
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
   for (int64_t bh = 0; bh < BH; ++bh) {
     double lam = (double)slopes[bh % H];
     double* Q = (double*)malloc(sizeof(double) * (size_t)(N * D + 1));
@@ -459,9 +463,9 @@ int la_oracle_backward_recurrent(const void* q, const void* k, const void* v, co
   int rc = bad_args(q, k, v, slopes, dq, B, H, N, D, E);
   if (rc) return rc;
   if (bad_grads(dout, dq, dk, dv)) return 1;
-  set_threads(nthreads);
+  const int nt = pick_threads(nthreads);
   int64_t BH = B * H;
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
   for (int64_t bh = 0; bh < BH; ++bh) {
     double gamma = exp(-(double)slopes[bh % H]);
     double* T = (double*)calloc((size_t)(E * D), sizeof(double));
@@ -527,9 +531,9 @@ int la_oracle_fused_layer(const void* q, const void* k, const void* v, const voi
   int rc = bad_args(q, k, v, slopes, out, B, H, N, D, E);
   if (rc) return rc;
   if (!gate || !norm_w || !(eps >= 0.0)) return 1;
-  set_threads(nthreads);
+  const int nt = pick_threads(nthreads);
   int64_t BH = B * H;
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
   for (int64_t bh = 0; bh < BH; ++bh) {
     int64_t h = bh % H;
     double gamma = exp(-(double)slopes[h]);
