@@ -150,6 +150,12 @@ def test_backward_and_anticausal_validation(lib):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_NULL
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 128, 128, None) == LA_ERR_SHAPE
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 96, 128, None) == LA_ERR_UNSUPPORTED
+    # every pointer is checked before the first launch (q and dk, dv are not
+    # operands of the dq launch)
+    assert f(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_NULL
+    assert f(FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 128, 128, None) == LA_ERR_ALIGN
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8, 1, 1, 8, 128, 128, None) == LA_ERR_ALIGN
     g = lib.lightning_attn_fwd_anticausal
     assert g(None, FAKE, FAKE, FAKE, None, None, FAKE, 1, 1, 8, 128, 128, 0, None) == LA_ERR_NULL
     assert g(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 1, 8, 128, 128, 100, None) == LA_ERR_SHAPE

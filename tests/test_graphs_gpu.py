@@ -70,6 +70,44 @@ def test_prefill_graph_replays_with_new_inputs(B, H, N, mode, noalloc):
     del graph
 
 
+@pytest.mark.parametrize("B,H,N", [(2, 80, 600), (1, 64, 2000), (1, 4, 3000)])
+def test_backward_graph_replays_with_new_inputs(B, H, N):
+    """The backward pass (dq launch + paired dk/dv launch, each role with its own
+    cleared control block) captured once and replayed with fresh inputs."""
+    q, k, v, g = (torch.empty((B, H, N, 128), dtype=torch.bfloat16, device=DEV) for _ in range(4))
+    dq, dk, dv = (torch.empty((B, H, N, 128), dtype=torch.float32, device=DEV) for _ in range(3))
+    sl_host = I.alibi_slopes(H)
+    sl = torch.from_numpy(sl_host).to(DEV)
+    call = lambda: ops.bwd(q, k, v, g, sl, dq, dk, dv)
+
+    def fill(seed):
+        host = _fill((q, k, v), B, H, N, 10 + seed)
+        gh = I.f32_to_bf16_bits(np.random.default_rng(seed).standard_normal((B, H, N, 128))
+                                .astype(np.float32))
+        g.copy_(torch.from_numpy(gh.view(np.int16)).view(torch.bfloat16))
+        return (*host, gh)
+
+    fill(0)
+    call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    for seed in (1, 2):
+        hq, hk, hv, hg = fill(seed)
+        for t in (dq, dk, dv):
+            t.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert ops.device_status(reset=True) == 0
+        for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv),
+                                  oracle.backward(hq, hk, hv, hg, sl_host)):
+            a = got.cpu().numpy()
+            assert np.isfinite(a).all(), (seed, name)
+            assert rel(a, ref) <= TOL_BF16, (seed, name)
+    del graph
+
+
 def _captured_node_types(call):
     """Node types of the graph that capturing call(stream) records."""
     from cuda.bindings import runtime as rt
