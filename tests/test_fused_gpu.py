@@ -13,7 +13,8 @@ import torch
 import oracle
 from long_context_fwd_b200 import inputs as I
 from long_context_fwd_b200 import ops
-from parity import TOL_BF16, bf16_to_dev, f32_to_dev, rel, worst_head
+from parity import (TOL_BF16, bf16_to_dev, f32_to_dev, fill_heads_from_host, host_workers, rel,
+                    worst_head)
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -68,3 +69,41 @@ def test_fused_layer_eps_and_gate_ranges(eps, gate_scale):
     got = _run(raw, gate, w, sl, eps)
     ref = oracle.fused_layer(*raw, gate, sl, w, eps)
     assert rel(got, ref) <= TOL_BF16
+
+
+def test_fused_layer_32k_workload_shapes_sampled_sequences():
+    """The fused layer on the benchmark's shapes (B=4, H=64, N=32768, lambda = 0
+    on heads h % 8 == 7; raw q, k, v and the gate ~ N(0, 1) drawn per sequence
+    on the host; one launch as the benchmark times it): the outputs of 12
+    sequences -- four lambda = 0 heads and eight decaying ones in the first and
+    last batch rows -- in full against the oracle."""
+    w = I.PREFILL_32K
+    sl = I.slopes_for(w)
+    nw = (1.0 + 0.25 * np.random.default_rng(77).standard_normal((w.H, w.E))).astype(np.float32)
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    checked = {(b, h) for b in (0, 3) for h in (7, 15, 0, 20, 41, 62)}
+    assert sum(sl[h] == 0.0 for _, h in checked) == 4
+
+    def draw(b, h):
+        rng = np.random.default_rng(7000 + b * w.H + h)
+        return tuple(I.f32_to_bf16_bits(rng.standard_normal((w.N, 128)).astype(np.float32))
+                     for _ in range(4))
+
+    def reference(b, h, hq, hk, hv, hg):
+        if (b, h) not in checked:
+            return None
+        return oracle.fused_layer(hq[None, None], hk[None, None], hv[None, None], hg[None, None],
+                                  sl[h:h + 1], nw[h:h + 1], 1e-6, threads=1)[0, 0]
+
+    q, k, v, g = (torch.empty((w.B, w.H, w.N, 128), dtype=torch.bfloat16, device=DEV)
+                  for _ in range(4))
+    refs = fill_heads_from_host(draw, (q, k, v, g), heads, reference, host_workers(0.3e9))
+    out = ops.fwd_fused(q, k, v, g, f32_to_dev(sl, DEV), f32_to_dev(nw, DEV), 1e-6)
+    torch.cuda.synchronize()
+    assert ops.device_status(reset=True) == 0
+    del q, k, v, g
+    for (b, h) in sorted(checked):
+        got = out[b, h].float().cpu().numpy()
+        assert np.isfinite(got).all(), (b, h)
+        assert rel(got, refs[(b, h)]) <= TOL_BF16, (b, h)
+    assert torch.isfinite(out).all()

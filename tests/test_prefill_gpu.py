@@ -329,21 +329,34 @@ def test_bf16_prefill_32k_workload_every_sequence():
 def test_bf16_prefill_1m_workload_every_head_sampled():
     """B=1, H=64, N=1,048,576, as the benchmark runs it, every head's inputs drawn
     on the host: each of the 64 heads checked at the 64 sampled positions against
-    the oracle's recurrence over all 1,048,576 tokens."""
+    the oracle's recurrence over all 1,048,576 tokens; and the state pass alone
+    (lightning_attn_state, as the benchmark's state leg runs it) on the same
+    inputs, four heads' states after the whole sequence against the oracle's."""
     w = I.PREFILL_1M
     sl = I.slopes_for(w)
     pos = I.sample_positions(w.N)
+    state_heads = (0, 21, 42, 63)
     q, k, v = (torch.empty((w.B, w.H, w.N, 128), dtype=torch.bfloat16, device=DEV)
                for _ in range(3))
+
+    def reference(b, h, hq, hk, hv):
+        args = (hq[None, None], hk[None, None], hv[None, None], sl[h:h + 1])
+        sampled = oracle.recurrent_sampled(*args, pos, threads=1)[0, 0]
+        if h not in state_heads:
+            return sampled, None
+        return sampled, oracle.recurrent(*args, return_state=True, threads=1)[1][0, 0]
+
     refs = fill_heads_from_host(
         lambda b, h: I.head_inputs(w, b, h), (q, k, v), [(0, h) for h in range(w.H)],
-        lambda b, h, hq, hk, hv: oracle.recurrent_sampled(
-            hq[None, None], hk[None, None], hv[None, None], sl[h:h + 1], pos, threads=1)[0, 0],
-        host_workers(2.5e9))
+        reference, host_workers(2.5e9))
     out = ops.fwd(q, k, v, f32_to_dev(sl, DEV))
+    states = ops.state(k, v, f32_to_dev(sl, DEV))
     torch.cuda.synchronize()
     assert ops.device_status(reset=True) == 0
     del q, k, v
+    for h in state_heads:
+        assert rel(states[0, h].cpu().numpy(), refs[(0, h)][1]) <= TOL_BF16, h
+    refs = {key: r[0] for key, r in refs.items()}
     got = out[0].index_select(1, torch.as_tensor(pos, device=DEV)).cpu().numpy()  # [H, 64, E]
     ref = np.stack([refs[(0, h)] for h in range(w.H)])
     for h in range(w.H):
