@@ -113,7 +113,9 @@ enum BarId : int {
   B_P1E = 35,  // phase 1: pair slot free again (3)
   B_KT = 38,   // phase 1: decayed K tile of a pair slot ready (3)
   B_ACT = 41,  // fused layer: Q and K tiles of a block activated (2)
-  B_COUNT = 43
+  B_CHAIN = 43,      // split scan: the entering chain listed and its pieces published
+  B_CHAIN_DONE = 44, // split scan: group X has combined the entering state
+  B_COUNT = 45
 };
 
 // Optional event trace (compiled only with -DLA_TRACE): %globaltimer stamps of
@@ -600,7 +602,58 @@ __device__ void mma_issuer(const Ctx& c, const Params& p) {
 }
 
 // ---------------------------------------------------------------------------
-// Group X: decay-causal mask and the in-place operand decays.
+// fp32 rows of 32 columns to and from global memory (states).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ld_global32(const float* src, uint32_t (&x)[32]) {
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 v = __ldcg(s4 + i);
+    x[4 * i] = __float_as_uint(v.x);
+    x[4 * i + 1] = __float_as_uint(v.y);
+    x[4 * i + 2] = __float_as_uint(v.z);
+    x[4 * i + 3] = __float_as_uint(v.w);
+  }
+}
+
+__device__ __forceinline__ void st_global32(float* dst, const uint32_t (&x)[32]) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    __stcg(d4 + i, make_float4(__uint_as_float(x[4 * i]), __uint_as_float(x[4 * i + 1]),
+                               __uint_as_float(x[4 * i + 2]), __uint_as_float(x[4 * i + 3])));
+}
+
+// Chunk states in the scan scratch use a thread-blocked layout: the float4 that
+// thread (row r, half hf) holds as its i-th vector of pass h lives at float4
+// index ((hf * 2 + h) * 8 + i) * 128 + r, so each warp-wide access covers 512
+// contiguous bytes.
+__device__ __forceinline__ void ld_scan32(const float* base, uint32_t r, uint32_t hf, uint32_t h,
+                                          uint32_t (&x)[32]) {
+  const float4* s4 = reinterpret_cast<const float4*>(base);
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i) {
+    const float4 v = __ldcg(s4 + ((hf * 2u + h) * 8u + i) * 128u + r);
+    x[4 * i] = __float_as_uint(v.x);
+    x[4 * i + 1] = __float_as_uint(v.y);
+    x[4 * i + 2] = __float_as_uint(v.z);
+    x[4 * i + 3] = __float_as_uint(v.w);
+  }
+}
+
+__device__ __forceinline__ void st_scan32(float* base, uint32_t r, uint32_t hf, uint32_t h,
+                                          const uint32_t (&x)[32]) {
+  float4* d4 = reinterpret_cast<float4*>(base);
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i)
+    __stcg(d4 + ((hf * 2u + h) * 8u + i) * 128u + r,
+           make_float4(__uint_as_float(x[4 * i]), __uint_as_float(x[4 * i + 1]),
+                       __uint_as_float(x[4 * i + 2]), __uint_as_float(x[4 * i + 3])));
+}
+
+// ---------------------------------------------------------------------------
+// Group X: decay-causal mask, the in-place operand decays and the split
+// scan's chained entering states.
 // ---------------------------------------------------------------------------
 template <bool REV, bool FUSED>
 __device__ void group_x(const Ctx& c, const Params& p) {
@@ -610,7 +663,55 @@ __device__ void group_x(const Ctx& c, const Params& p) {
   const uint32_t hf = warp >> 2;
   const uint32_t lane_base = ((warp & 3u) * 32u) << 16;
   const uint32_t gtab = c.sbase + OFF_GTAB;
-  uint32_t q_it = 0, k_it = 0, w_it = 0, gb = 0, xs_n = 0, p1_it = 0;
+  uint32_t q_it = 0, k_it = 0, w_it = 0, gb = 0, xs_n = 0, p1_it = 0, chain_n = 0;
+  // Split scan: an output item that starts inside its sequence enters with
+  //   S(X) = gamma^(128 (X - x_lo)) S(x_lo) + sum_j gamma^(128 (X - y_j)) piece_j
+  // over the published pieces that group Y's first warp has listed and seen.
+  // Group X combines it (the MMA issuer waits for the state anyway): two column
+  // quarters of row r per thread, half of what each of group Y's threads would
+  // load, into the state's bf16 copy and the TMEM state.
+  auto combine_chain = [&](const Item& it, float lam) -> bool {
+    if (!cwait(c, p, B_CHAIN, chain_n++ & 1u)) return false;
+    const int n = static_cast<int>(c.misc[18]);
+    const int64_t span = it.t0 / BLK;  // X - x_lo, in blocks
+    const float g_all = expf(-lam * static_cast<float>(span * BLK));
+    const float g0 = expf(-lam * static_cast<float>(min(BLK, it.Lc)));
+    const float* init = p.init_state && static_cast<int>(r) < p.D
+                            ? p.init_state + static_cast<int64_t>(it.seq) * p.D * p.E +
+                                  static_cast<int64_t>(r) * p.E
+                            : nullptr;
+    const float* prefix = cta_role(p) ? p.prefix1 : p.prefix;
+    const uint32_t t_kv = c.tmem + lane_base + TM_KV;
+#pragma unroll 1
+    for (uint32_t qq = 0; qq < 2; ++qq) {
+      const uint32_t q = 2u * hf + qq;
+      uint32_t prev[32];
+      if (init && 32 * static_cast<int>(q) < p.E) {
+        ld_global32(init + 32 * q, prev);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) prev[i] = 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) prev[i] = __float_as_uint(g_all * __uint_as_float(prev[i]));
+#pragma unroll 1
+      for (int j = 0; j < n; ++j) {
+        uint32_t part[32];
+        ld_scan32(prefix + static_cast<int64_t>(c.chain[2 * j]) * (HD * HD), r, q >> 1, q & 1u, part);
+        const float w = expf(-lam * static_cast<float>(static_cast<int>(c.chain[2 * j + 1]) * BLK));
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          prev[i] = __float_as_uint(fmaf(w, __uint_as_float(part[i]), __uint_as_float(prev[i])));
+      }
+      store_half_bf16(c.sbase + OFF_KVB + hf * PLANE + r * 128u, r, qq, prev, 1.f);
+      tmem_st32_scaled(t_kv + 32u * q, prev, g0);
+    }
+    fence_proxy_async_smem();
+    tmem_wait_st();
+    tc_fence_before();
+    warp_arrive(&c.bar[B_CHAIN_DONE]);
+    return true;
+  };
   // fused layer: SiLU on the Q and K tiles of phase-2 block gidx in place, then
   // the MMA issuer may compute their scores
   auto activate_qk = [&](uint32_t qi, uint32_t ki, uint32_t gidx) -> bool {
@@ -639,7 +740,8 @@ __device__ void group_x(const Ctx& c, const Params& p) {
     if (!gsync(c, p, B_XSYNC, xs_n)) break;
 
     bool ok = true;
-    if (it.phase1) {  // K rows decayed to the chunk end: gamma^(Lc-1-j)
+    if (it.enter && p.mode == MODE_SPLIT_SCAN) ok = combine_chain(it, lam);
+    if (it.phase1 && ok) {  // K rows decayed to the chunk end: gamma^(Lc-1-j)
       for (int b = 0; b < it.nb && ok; ++b) {
         const uint32_t slot = p1_it % P1_SLOTS;
         if (!cwait(c, p, B_P1F + slot, (p1_it / P1_SLOTS) & 1u)) { ok = false; break; }
@@ -752,55 +854,8 @@ __device__ void group_x(const Ctx& c, const Params& p) {
 }
 
 // ---------------------------------------------------------------------------
-// Group Y: state copy/decay, chunk scan, epilogue.
+// Group Y: entering states, state copy/decay, chunk scan, epilogue.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void ld_global32(const float* src, uint32_t (&x)[32]) {
-  const float4* s4 = reinterpret_cast<const float4*>(src);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 v = __ldcg(s4 + i);
-    x[4 * i] = __float_as_uint(v.x);
-    x[4 * i + 1] = __float_as_uint(v.y);
-    x[4 * i + 2] = __float_as_uint(v.z);
-    x[4 * i + 3] = __float_as_uint(v.w);
-  }
-}
-
-__device__ __forceinline__ void st_global32(float* dst, const uint32_t (&x)[32]) {
-  float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    __stcg(d4 + i, make_float4(__uint_as_float(x[4 * i]), __uint_as_float(x[4 * i + 1]),
-                               __uint_as_float(x[4 * i + 2]), __uint_as_float(x[4 * i + 3])));
-}
-
-// Chunk states in the scan scratch use a thread-blocked layout: the float4 that
-// thread (row r, half hf) holds as its i-th vector of pass h lives at float4
-// index ((hf * 2 + h) * 8 + i) * 128 + r, so each warp-wide access covers 512
-// contiguous bytes.
-__device__ __forceinline__ void ld_scan32(const float* base, uint32_t r, uint32_t hf, uint32_t h,
-                                          uint32_t (&x)[32]) {
-  const float4* s4 = reinterpret_cast<const float4*>(base);
-#pragma unroll
-  for (uint32_t i = 0; i < 8; ++i) {
-    const float4 v = __ldcg(s4 + ((hf * 2u + h) * 8u + i) * 128u + r);
-    x[4 * i] = __float_as_uint(v.x);
-    x[4 * i + 1] = __float_as_uint(v.y);
-    x[4 * i + 2] = __float_as_uint(v.z);
-    x[4 * i + 3] = __float_as_uint(v.w);
-  }
-}
-
-__device__ __forceinline__ void st_scan32(float* base, uint32_t r, uint32_t hf, uint32_t h,
-                                          const uint32_t (&x)[32]) {
-  float4* d4 = reinterpret_cast<float4*>(base);
-#pragma unroll
-  for (uint32_t i = 0; i < 8; ++i)
-    __stcg(d4 + ((hf * 2u + h) * 8u + i) * 128u + r,
-           make_float4(__uint_as_float(x[4 * i]), __uint_as_float(x[4 * i + 1]),
-                       __uint_as_float(x[4 * i + 2]), __uint_as_float(x[4 * i + 3])));
-}
-
 template <int RANK, bool REV, bool FUSED>
 __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
   const uint32_t t = threadIdx.x - 32u * Y_WARP0;  // 0..127
@@ -815,7 +870,7 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
   const int64_t state_elems = static_cast<int64_t>(p.D) * p.E;
   const bool leader = (t == 0);
   const uint64_t pol_out = policy_evict_first();
-  uint32_t v_it = 0, w_it = 0, gb = 0, agg_n = 0, ys_n = 0;
+  uint32_t v_it = 0, w_it = 0, gb = 0, agg_n = 0, ys_n = 0, chain_done_n = 0;
   // this CTA's scratch and plain-store output (the second role's in a paired launch)
   const bool role1 = cta_role(p) != 0;
   float* const prefix = role1 ? p.prefix1 : p.prefix;
@@ -884,6 +939,8 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
             break;
           }
         }
+        // group X combines a chain (it waits for the list and the flags)
+        if (chain && t == 0) mbar_arrive(&c.bar[B_CHAIN]);
       }
       if (!gsync(c, p, B_YSYNC, ys_n)) break;
       if (!chain) scan_src = prefix + static_cast<int64_t>(it.enter_slot) * (HD * HD);
@@ -891,13 +948,16 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
     // the caller's initial state enters at block 0 of a sequence (or through
     // the chain); never into a local state -- except in the state pass, where
     // the first chunk's inclusive state starts from it
-    if (p.init_state && (it.p2 || p.state_only) && (!it.enter || chain) && row_in)
+    if (p.init_state && (it.p2 || p.state_only) && !it.enter && row_in)
       init_src = p.init_state + static_cast<int64_t>(it.seq) * state_elems + row_off;
     if (leader) LA_TRACE_EVENT(16, w_it);
     if (it.phase1 && !cwait(c, p, B_AGG_FULL, agg_n++ & 1u)) break;
     if (leader) LA_TRACE_EVENT(17, w_it);
-    tc_fence_after();
-    {
+    if (chain) {  // group X has combined the entering state into KVB and TMEM
+      if (!cwait(c, p, B_CHAIN_DONE, chain_done_n++ & 1u)) break;
+      tc_fence_after();
+    } else {
+      tc_fence_after();
       const float gL = expf(-lam * static_cast<float>(it.Lc));
       const float g0 = expf(-lam * static_cast<float>(min(BLK, it.Lc)));
       float* pub = prefix + static_cast<int64_t>(it.pub_slot) * (HD * HD);
@@ -911,22 +971,6 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) prev[i] = 0u;
-        }
-        if (chain) {
-          // S(X) = gamma^(128 (X - x_lo)) S(x_lo) + sum_j gamma^(128 (X - y_j)) piece_j
-          const int n = static_cast<int>(c.misc[18]);
-          const float g_all = expf(-lam * static_cast<float>((x_hi - x_lo) * BLK));
-#pragma unroll
-          for (int i = 0; i < 32; ++i) prev[i] = __float_as_uint(g_all * __uint_as_float(prev[i]));
-#pragma unroll 1
-          for (int j = 0; j < n; ++j) {
-            uint32_t part[32];
-            ld_scan32(prefix + static_cast<int64_t>(c.chain[2 * j]) * (HD * HD), r, q >> 1, q & 1u, part);
-            const float w = expf(-lam * static_cast<float>(static_cast<int>(c.chain[2 * j + 1]) * BLK));
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              prev[i] = __float_as_uint(fmaf(w, __uint_as_float(part[i]), __uint_as_float(prev[i])));
-          }
         }
         if (it.phase1) {
           uint32_t agg[32];
@@ -1228,6 +1272,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&c.bar[B_KT + i], X_WARPS);
     }
     mbar_init(&c.bar[B_READY], X_WARPS);
+    mbar_init(&c.bar[B_CHAIN], 1);
+    mbar_init(&c.bar[B_CHAIN_DONE], X_WARPS);
     mbar_init(&c.bar[B_KVB_READY], Y_WARPS);
     mbar_init(&c.bar[B_KVO_DONE], 1);
     mbar_init(&c.bar[B_O_FULL], 1);
