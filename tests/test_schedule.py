@@ -69,7 +69,9 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("sms", [148, 132, 160])
+# 74 and 66: each role of the backward's paired launch is planned for half the
+# CTAs of a 148- or 132-SM part
+@pytest.mark.parametrize("sms", [148, 132, 160, 74, 66])
 @pytest.mark.parametrize("B,H,N", SHAPES)
 def test_every_output_once(B, H, N, sms):
     info, items = _plan(B, H, N, sms=sms)
@@ -137,7 +139,7 @@ def _check_handover(B, H, N, sms, info, items):
         assert info["slots"] == 0 and not any(it["flags"] & (ENTER | PUBLISH) for it in items)
 
 
-@pytest.mark.parametrize("sms", [148, 132])
+@pytest.mark.parametrize("sms", [148, 132, 74])
 @pytest.mark.parametrize("B,H,N", [(4, 64, 32768), (1, 149, 1025), (2, 80, 1100), (1, 150, 2500),
                                    (1, 296, 300), (3, 100, 700), (1, 200, 5000)])
 def test_balanced_handover(B, H, N, sms):
@@ -145,7 +147,7 @@ def test_balanced_handover(B, H, N, sms):
     _check_handover(B, H, N, sms, info, items)
 
 
-@pytest.mark.parametrize("sms", [148, 132, 160])
+@pytest.mark.parametrize("sms", [148, 132, 160, 74, 66])
 @pytest.mark.parametrize("B,H,N", [(1, 64, 8192), (1, 64, 1048576), (1, 19, 3000), (1, 37, 1025),
                                    (1, 100, 2000), (1, 147, 1200), (1, 64, 1152),
                                    (1, 20, 100000), (2, 40, 9000)])
