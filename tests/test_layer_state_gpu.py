@@ -191,3 +191,26 @@ def test_decode_layer_strided_output_rows():
     assert rel(outv.float().cpu().numpy(), ref[:, :, 0]) <= TOL_BF16
     assert torch.all(wide[:, 1::2] == 0)
     assert rel(state.cpu().numpy(), sref) <= 1e-4
+
+
+@pytest.mark.parametrize("D,E", [(64, 128), (128, 64), (128, 128)])
+def test_split_scan_layer_with_state(D, E):
+    """The fused layer in the split scan (64 sequences on the grid), entering
+    from a caller's state: the items that start inside a sequence combine that
+    state with the chained pieces (group X's combine, including the rows and
+    columns past 64-wide heads), and the final state is handed back."""
+    B, H, N = 1, 64, 2500
+    sms = torch.cuda.get_device_properties(DEV).multi_processor_count
+    assert ops.fwd_plan(B, H, N, 0, sms)[0]["mode"] == 2
+    q, k, v, g, w, sl = _case(B, H, N, D, E, seed=60 + D + E)
+    s0 = 0.05 * np.random.default_rng(D + 2 * E).standard_normal((B, H, D, E))
+    fin = torch.zeros((B, H, D, E), dtype=torch.float32, device=DEV)
+    out = ops.fwd_fused_ex(*(bf16_to_dev(x, DEV) for x in (q, k, v, g)), f32_to_dev(sl, DEV),
+                           f32_to_dev(w, DEV), 1e-6, init_state=f32_to_dev(s0.astype(np.float32), DEV),
+                           final_state=fin)
+    _done()
+    ref, sref = oracle.fused_layer(q, k, v, g, sl, w, 1e-6, s0=s0, return_state=True)
+    got = out.float().cpu().numpy()
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+    assert rel(fin.cpu().numpy(), sref) <= TOL_BF16
