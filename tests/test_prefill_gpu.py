@@ -189,6 +189,25 @@ def test_bf16_split_scan_initial_and_final_state():
     assert worst_head(fin.cpu().numpy(), sref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("D,E", [(64, 128), (128, 64), (64, 64)])
+def test_bf16_split_scan_narrow_heads_with_state(D, E):
+    """The split scan's chained entering states from a caller's initial state
+    on 64-wide heads (rows or columns of the 128 x 128 state past D or E stay
+    zero), with the final state handed back."""
+    B, H, N = 1, 64, 2200
+    w = I.Workload(f"splitnarrow{D}{E}", B, H, N, D, E, "bf16", index=1900 + D + E)
+    q, k, v = I.prefill_inputs(w)
+    sl = I.alibi_slopes(H)
+    sl[4::9] = 0.0
+    s0 = (np.random.default_rng(D * E).standard_normal((B, H, D, E)) * 0.05).astype(np.float32)
+    fin = torch.zeros((B, H, D, E), dtype=torch.float32, device=DEV)
+    got = _run(q, k, v, sl, init_state=f32_to_dev(s0, DEV), final_state=fin)
+    ref, sref = oracle.recurrent(q, k, v, sl, s0=s0.astype(np.float64), return_state=True)
+    assert rel(got, ref) <= TOL_BF16
+    assert worst_head(got, ref) <= TOL_BF16
+    assert rel(fin.cpu().numpy(), sref) <= TOL_BF16
+
+
 # D != E on the tensor-core path: 64-wide q/k or v run on the 128-wide tiles
 # with the missing columns zero-filled by the tensor maps.  Whole sequences,
 # explicit chunks, the split scan and the hand-over; ragged ends.
