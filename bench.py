@@ -796,7 +796,8 @@ def main_ours(args):
                                                      bf16, None, peak_src)}
     if bwd:
         # minimal traffic of the operation: q, k, v, dout read once (bf16), dq,
-        # dk, dv written once (fp32); flops: three launches of the blocked form
+        # dk, dv written once (fp32); flops: three operators in the blocked form
+        # (dq, dk, dv, whether dk and dv share a launch or not)
         units = w.B * w.H * w.N
         bytes_min = units * (2 * (2 * w.D + 2 * w.E) + 4 * (2 * w.D + w.E))
         r = roofline(bytes_min, 3 * prefill_flops(w), bwd["ms"], hbm, bf16, None, peak_src)
