@@ -119,6 +119,9 @@ def parse():
                     help="prefill q/k/v/out layout: [B][H][N][D] or [B][N][H][D]")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the end-to-end leg")
+    ap.add_argument("--e2e-groups", type=int, default=16,
+                    help="groups of sequences the end-to-end step pipelines (largest divisor "
+                         "of B*H not above it that splits whole rows or equal runs of heads)")
     ap.add_argument("--e2e-upload-streams", type=int, default=1,
                     help="streams the end-to-end leg's uploads alternate between (two measured "
                          "slower: 146 vs 134-136 ms per step)")
@@ -390,7 +393,7 @@ def bench_prefill(args, dist, w, dev):
     # it is computed, so uploads run continuously and overlap the downloads
     # (PCIe is full duplex).
     nseq = w.B * w.H
-    G = next((g for g in (16, 8, 4, 2) if nseq % g == 0 and
+    G = next((g for g in range(min(args.e2e_groups, nseq), 1, -1) if nseq % g == 0 and
               (w.H % (nseq // g) == 0 or (nseq // g) % w.H == 0)), 1)
     per = nseq // G
     ups = [torch.cuda.Stream(device=dev) for _ in range(max(1, args.e2e_upload_streams))]
