@@ -939,7 +939,9 @@ __device__ void group_y(const Ctx& c, const Params& p, const CUtensorMap* to) {
             break;
           }
         }
-        // group X combines a chain (it waits for the list and the flags)
+        // group X combines a chain (it waits for the list and the flags): the
+        // warp barrier orders every lane's acquire before lane 0's release
+        __syncwarp();
         if (chain && t == 0) mbar_arrive(&c.bar[B_CHAIN]);
       }
       if (!gsync(c, p, B_YSYNC, ys_n)) break;
