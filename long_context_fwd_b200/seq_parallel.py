@@ -34,11 +34,13 @@ import torch.distributed as dist
 class Steps(NamedTuple):
     """The three compute steps: state(k, v, slopes) -> [B,H,D,E];
     combine(states [R,B,H,D,E], counts, slopes, init_state) -> [B,H,D,E];
-    prefill(q, k, v, slopes, init_state) -> out [B,H,N,E]."""
+    prefill(q, k, v, slopes, init_state) -> out [B,H,N,E]; and the dtype of
+    the states and outputs they return (an empty chunk's are made in it)."""
 
     state: Callable
     combine: Callable
     prefill: Callable
+    dtype: torch.dtype = torch.float32
 
 
 def cuda_steps() -> Steps:
@@ -58,15 +60,21 @@ def prefill_sequence_parallel(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     """Prefill of this rank's chunk of every (b, h) sequence.
 
     q, k [B,H,n_r,D], v [B,H,n_r,E] hold tokens of chunk r = this rank's index
-    in ``group`` (chunks in rank order; lengths may differ between ranks).
-    init_state (optional, [B,H,D,E]) is the state before chunk 0, the same on
-    every rank.  Returns (out [B,H,n_r,E] of this chunk, the state after the
-    whole sequence [B,H,D,E]).  Every rank takes the same collective steps.
+    in ``group`` (chunks in rank order; lengths may differ between ranks, and
+    a rank's chunk may be empty).  init_state (optional, [B,H,D,E]) is the
+    state before chunk 0, the same on every rank.  Returns (out [B,H,n_r,E] of
+    this chunk, the state after the whole sequence [B,H,D,E]).  Every rank
+    takes the same collective steps.
     """
     steps = steps or cuda_steps()
     rank = dist.get_rank(group)
     world = dist.get_world_size(group)
-    local = steps.state(k, v, slopes).contiguous()
+    B, H, n_r, D = k.shape
+    E = v.shape[-1]
+    if n_r == 0:  # an empty chunk adds nothing to the state and has no outputs
+        local = torch.zeros((B, H, D, E), dtype=steps.dtype, device=k.device)
+    else:
+        local = steps.state(k, v, slopes).contiguous()
     parts = [torch.empty_like(local) for _ in range(world)]
     dist.all_gather(parts, local, group=group)
     n_local = torch.tensor([q.shape[2]], dtype=torch.int64, device=local.device)
@@ -75,6 +83,9 @@ def prefill_sequence_parallel(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     counts = [int(c.item()) for c in counts_t]
     states = torch.stack(parts)
     entering = steps.combine(states[:rank].contiguous(), counts[:rank], slopes, init_state)
-    out = steps.prefill(q, k, v, slopes, entering)
+    if n_r == 0:
+        out = torch.empty((B, H, 0, E), dtype=steps.dtype, device=k.device)
+    else:
+        out = steps.prefill(q, k, v, slopes, entering)
     final = steps.combine(states, counts, slopes, init_state)
     return out, final

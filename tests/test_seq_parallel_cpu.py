@@ -8,7 +8,8 @@ the float64 oracle (its recurrence for the state and the prefill, the
 linearity of the recurrence in its initial state for the combination), so
 that the ranks' chunk outputs, put together, must equal the oracle's
 recurrence over the whole sequence -- checking the collective order, the rank
-slicing and the uneven chunk lengths the module handles.
+slicing and the uneven chunk lengths the module handles (with four ranks, one
+chunk is empty).
 """
 import os
 import socket
@@ -29,7 +30,8 @@ def _free_port():
     return port
 
 
-CUTS = {2: (0, 700, 1500), 3: (0, 128, 1000, 1501)}
+CUTS = {2: (0, 700, 1500), 3: (0, 128, 1000, 1501),
+        4: (0, 300, 300, 1200, 1333)}  # rank 1's chunk is empty
 
 
 def _oracle_steps():
@@ -52,7 +54,7 @@ def _oracle_steps():
         return torch.from_numpy(oracle.recurrent(q.numpy(), k.numpy(), v.numpy(), sl.numpy(),
                                                  s0=init.numpy()))
 
-    return Steps(state, combine, prefill)
+    return Steps(state, combine, prefill, torch.float64)
 
 
 def _rank(rank, world, port, out):
@@ -77,7 +79,7 @@ def _rank(rank, world, port, out):
     dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 4])
 def test_ranks_chunks_equal_the_whole_sequence(world):
     import oracle
     from long_context_fwd_b200 import inputs as I
