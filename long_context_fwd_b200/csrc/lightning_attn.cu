@@ -933,7 +933,8 @@ int lightning_attn_state_combine(const float* states, int R, const int* chunk_to
   a.H = H;
   a.R = R;
   const int64_t blocks = (a.total4 + 255) / 256;
-  const int grid = static_cast<int>(blocks < 4 * 148 * 8 ? blocks : 4 * 148 * 8);
+  const int64_t cap = 32ll * sm_count();  // grid-stride loop: a few waves of 256 threads
+  const int grid = static_cast<int>(blocks < cap ? blocks : cap);
   la::state_combine_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
   return launch_status();
 }
